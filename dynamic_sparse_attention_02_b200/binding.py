@@ -1,0 +1,252 @@
+"""Thin ctypes binding over libminfer.so (include/minfer.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  Functions carry the C names; they take torch CUDA
+tensors (torch is used for device memory and streams), allocate outputs and
+workspace with torch when the caller does not pass them, and raise
+``MinferError`` on a non-zero status.  There is no fallback: if the library
+is missing or a CUDA call fails, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libminfer.so")
+
+MI_OK, MI_ERR_INVALID_ARG, MI_ERR_UNSUPPORTED, MI_ERR_WORKSPACE, MI_ERR_CUDA = range(5)
+MI_PATTERN_ASHAPE, MI_PATTERN_VS, MI_PATTERN_BS = 0, 1, 2
+MI_OP_VS_INDEX, MI_OP_BS_INDEX, MI_OP_VS_ATTN, MI_OP_BS_ATTN, MI_OP_ASHAPE_ATTN = 1, 2, 3, 4, 5
+MI_STAGE_START, MI_STAGE_INDEX_DONE, MI_STAGE_ATTN_DONE, MI_STAGE_EVENTS = 0, 1, 2, 3
+MI_MAX_HEADS = 256
+MI_BLOCK = 64
+
+# every symbol include/minfer.h declares
+EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
+           "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
+           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer"]
+
+
+class MinferError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = f"{fn}: {_lib_handle().mi_status_str(status).decode()} (status {status})"
+        if status == MI_ERR_CUDA:
+            msg += f", cudaError {_lib_handle().mi_last_cuda_error()}"
+        super().__init__(msg)
+
+
+class mi_params(ctypes.Structure):
+    _fields_ = [("last_q", ctypes.c_int), ("vertical_size", ctypes.c_int),
+                ("slash_size", ctypes.c_int), ("topk_blocks", ctypes.c_int),
+                ("sink", ctypes.c_int), ("window", ctypes.c_int)]
+
+
+_lib = None
+
+
+def _lib_handle():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run "
+                               "`python -m dynamic_sparse_attention_02_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.mi_status_str.argtypes = [I]
+        lib.mi_status_str.restype = ctypes.c_char_p
+        lib.mi_last_cuda_error.restype = I
+        lib.mi_version.restype = ctypes.c_char_p
+        lib.mi_workspace_bytes.argtypes = [I] * 10
+        lib.mi_workspace_bytes.restype = SZ
+        lib.mi_prefill_workspace_bytes.argtypes = [I, I, I, I, P, ctypes.POINTER(mi_params)]
+        lib.mi_prefill_workspace_bytes.restype = SZ
+        lib.mi_vs_index.argtypes = [P, P, I, I, I, I, F, I, I, I, P, I, P, P, P, P, P, SZ, P]
+        lib.mi_bs_index.argtypes = [P, P, I, I, I, I, F, I, I, P, I, P, P, P, SZ, P]
+        lib.mi_vs_sparse_attn.argtypes = [P, P, P, I, I, I, I, F, P, I, P, I, P, I, P, P, P, P,
+                                          SZ, P]
+        lib.mi_block_sparse_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, I, I, P, I, P, P, P,
+                                             P, SZ, P]
+        lib.mi_ashape_attn.argtypes = [P, P, P, I, I, I, I, F, I, I, P, I, P, P, P, P, SZ, P]
+        lib.mi_prefill_layer.argtypes = [P, P, P, I, I, I, I, F, P, ctypes.POINTER(mi_params),
+                                         P, P, P, P, SZ, P, P]
+        for name in EXPORTS[5:]:
+            getattr(lib, name).restype = I
+        _lib = lib
+    return _lib
+
+
+def lib():
+    """The loaded ctypes library (raises if it is not built)."""
+    return _lib_handle()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _heads(heads, Hq):
+    if heads is None:
+        return None, Hq, None
+    arr = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    return arr, int(arr.size), arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(fn, rc):
+    if rc != MI_OK:
+        raise MinferError(fn, rc)
+
+
+def _shape(q, k):
+    Hq, N, d = q.shape
+    return Hq, k.shape[0], N, d
+
+
+def _workspace(nbytes, device, ws):
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def mi_status_str(status: int) -> str:
+    return _lib_handle().mi_status_str(status).decode()
+
+
+def mi_version() -> str:
+    return _lib_handle().mi_version().decode()
+
+
+def mi_workspace_bytes(op, Hq, Hkv, N, d, n_heads=0, last_q=0, vertical_size=0, slash_size=0,
+                       topk_blocks=0) -> int:
+    return int(_lib_handle().mi_workspace_bytes(op, Hq, Hkv, N, d, n_heads, last_q,
+                                                vertical_size, slash_size, topk_blocks))
+
+
+def make_params(last_q=64, vertical_size=1000, slash_size=6096, topk_blocks=100, sink=64,
+                window=1024) -> mi_params:
+    return mi_params(last_q, vertical_size, slash_size, topk_blocks, sink, window)
+
+
+def mi_prefill_workspace_bytes(Hq, Hkv, N, d, pattern, params: mi_params) -> int:
+    pat = None if pattern is None else np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
+    pp = None if pat is None else pat.ctypes.data_as(ctypes.c_void_p)
+    return int(_lib_handle().mi_prefill_workspace_bytes(Hq, Hkv, N, d, pp, ctypes.byref(params)))
+
+
+def mi_vs_index(q, k, last_q, vertical_size, slash_size, heads: Optional[Sequence[int]] = None,
+                scale=0.0, ws=None, want_scores=False, stream=None):
+    """Vertical-Slash index: (v_idx, s_idx[, v_score, s_score]) per listed head."""
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    dev = q.device
+    v_idx = torch.empty(n, vertical_size, dtype=torch.int32, device=dev)
+    s_idx = torch.empty(n, slash_size, dtype=torch.int32, device=dev)
+    vs = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    ss = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    nb = mi_workspace_bytes(MI_OP_VS_INDEX, Hq, Hkv, N, d, n, last_q, vertical_size, slash_size)
+    ws = _workspace(nb, dev, ws)
+    rc = _lib_handle().mi_vs_index(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, last_q, vertical_size,
+                                   slash_size, hp, n, _ptr(v_idx), _ptr(s_idx), _ptr(vs), _ptr(ss),
+                                   _ptr(ws), ws.numel(), _stream(stream))
+    _check("mi_vs_index", rc)
+    return (v_idx, s_idx, vs, ss) if want_scores else (v_idx, s_idx)
+
+
+def mi_bs_index(q, k, topk, heads=None, scale=0.0, ws=None, stream=None):
+    """Block-Sparse index: (blk_idx [n, N/64, topk], blk_cnt [n, N/64])."""
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    dev = q.device
+    nB = N // MI_BLOCK
+    blk_idx = torch.empty(n, nB, topk, dtype=torch.int32, device=dev)
+    blk_cnt = torch.empty(n, nB, dtype=torch.int32, device=dev)
+    ws = _workspace(mi_workspace_bytes(MI_OP_BS_INDEX, Hq, Hkv, N, d, n), dev, ws)
+    rc = _lib_handle().mi_bs_index(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, MI_BLOCK, topk, hp, n,
+                                   _ptr(blk_idx), _ptr(blk_cnt), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+    _check("mi_bs_index", rc)
+    return blk_idx, blk_cnt
+
+
+def _attn_out(q, out, lse, want_lse):
+    if out is None:
+        out = torch.zeros_like(q)
+    if lse is None and want_lse:
+        lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def mi_vs_sparse_attn(q, k, v, v_idx, s_idx, heads=None, scale=0.0, out=None, lse=None,
+                      want_lse=True, err_count=None, ws=None, stream=None):
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse)
+    kv = v_idx.shape[-1] if v_idx is not None else 0
+    ks = s_idx.shape[-1] if s_idx is not None else 0
+    ws = _workspace(mi_workspace_bytes(MI_OP_VS_ATTN, Hq, Hkv, N, d, n, 0, kv, ks), q.device, ws)
+    rc = _lib_handle().mi_vs_sparse_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
+                                         _ptr(v_idx), kv, _ptr(s_idx), ks, hp, n, _ptr(out),
+                                         _ptr(lse), _ptr(err_count), _ptr(ws), ws.numel(),
+                                         _stream(stream))
+    _check("mi_vs_sparse_attn", rc)
+    return out, lse
+
+
+def mi_block_sparse_attn(q, k, v, blk_idx, blk_cnt, heads=None, scale=0.0, out=None, lse=None,
+                         want_lse=True, err_count=None, stream=None):
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse)
+    topk = blk_idx.shape[-1]
+    rc = _lib_handle().mi_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
+                                            _ptr(blk_idx), _ptr(blk_cnt), topk, MI_BLOCK, hp, n,
+                                            _ptr(out), _ptr(lse), _ptr(err_count), None, 0,
+                                            _stream(stream))
+    _check("mi_block_sparse_attn", rc)
+    return out, lse
+
+
+def mi_ashape_attn(q, k, v, sink, window, heads=None, scale=0.0, out=None, lse=None,
+                   want_lse=True, err_count=None, stream=None):
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse)
+    rc = _lib_handle().mi_ashape_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, sink,
+                                      window, hp, n, _ptr(out), _ptr(lse), _ptr(err_count), None,
+                                      0, _stream(stream))
+    _check("mi_ashape_attn", rc)
+    return out, lse
+
+
+def mi_prefill_layer(q, k, v, pattern, params: mi_params, scale=0.0, out=None, lse=None,
+                     want_lse=False, err_count=None, ws=None, stage_events=None, stream=None):
+    """One layer: per-head pattern table (host int8 [Hq]) -> index + sparse attention."""
+    Hq, Hkv, N, d = _shape(q, k)
+    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
+    out, lse = _attn_out(q, out, lse, want_lse)
+    ws = _workspace(mi_prefill_workspace_bytes(Hq, Hkv, N, d, pat, params), q.device, ws)
+    ev = None
+    if stage_events is not None:
+        for e in stage_events:
+            if not e.cuda_event:  # torch creates the CUDA event on first record
+                e.record()
+        ev = (ctypes.c_void_p * MI_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
+    rc = _lib_handle().mi_prefill_layer(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
+                                        pat.ctypes.data_as(ctypes.c_void_p), ctypes.byref(params),
+                                        _ptr(out), _ptr(lse), _ptr(err_count), _ptr(ws),
+                                        ws.numel(), _stream(stream), ev)
+    _check("mi_prefill_layer", rc)
+    return out, lse

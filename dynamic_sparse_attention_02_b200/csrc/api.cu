@@ -1,0 +1,374 @@
+// api.cu -- the C ABI declared in include/minfer.h: argument validation on
+// the host (nothing is launched when a check fails), workspace carving, and
+// the per-head pattern dispatcher of mi_prefill_layer (aifetchly guide,
+// "Phase 2: The Online Dynamic Kernel Router": each head goes to the kernel
+// of its offline-assigned pattern, with no host-device synchronisation).
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+using namespace minfer;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MI_OK;
+    g_last_cuda_error = (int)e;
+    return MI_ERR_CUDA;
+}
+
+// Shapes every entry point shares.  Fills `hl` with the listed heads
+// (pattern and per-pattern position filled by the caller).
+int check_shapes(const void* q, const void* k, int Hq, int Hkv, int N, int d,
+                 const int32_t* heads, int n_heads, HeadList& hl) {
+    if (!q || !k) return MI_ERR_INVALID_ARG;
+    if (Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || n_heads < 0) return MI_ERR_INVALID_ARG;
+    if (Hq % Hkv) return MI_ERR_INVALID_ARG;
+    if (Hq > MI_MAX_HEADS) return MI_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return MI_ERR_UNSUPPORTED;
+    if (N % MI_BLOCK) return MI_ERR_UNSUPPORTED;
+    if ((long long)Hq * N >= (1LL << 31) || N > (1 << 24)) return MI_ERR_UNSUPPORTED;
+    hl.n = 0;
+    if (!heads) {
+        for (int h = 0; h < Hq; ++h) hl.e[hl.n++] = pack_head(h, 0, h);
+        return MI_OK;
+    }
+    if (n_heads > Hq) return MI_ERR_INVALID_ARG;
+    bool seen[MI_MAX_HEADS] = {};
+    for (int i = 0; i < n_heads; ++i) {
+        const int h = heads[i];
+        if (h < 0 || h >= Hq || seen[h]) return MI_ERR_INVALID_ARG;
+        seen[h] = true;
+        hl.e[hl.n++] = pack_head(h, 0, i);
+    }
+    return MI_OK;
+}
+
+void set_pattern(HeadList& hl, int pattern) {
+    for (int i = 0; i < hl.n; ++i) hl.e[i] = pack_head(head_qh(hl.e[i]), pattern, i);
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (need == 0) return MI_OK;
+    if (!ws || ws_bytes < need) return MI_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return MI_ERR_WORKSPACE;
+    return MI_OK;
+}
+
+double eff_scale(float scale, int d) {
+    return scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+}
+
+int check_vs_params(int N, int last_q, int vertical_size, int slash_size) {
+    if (last_q <= 0 || vertical_size < 0 || slash_size < 0) return MI_ERR_INVALID_ARG;
+    if (last_q > N || last_q > 1024) return MI_ERR_UNSUPPORTED;
+    return MI_OK;
+}
+
+size_t vs_index_bytes(int n, int N, int L) {
+    WsCarver c(nullptr);
+    carve_vs_index(c, n, N, L, true, true);
+    return c.bytes();
+}
+size_t bs_index_bytes(int n, int Hkv, int N, int d) {
+    WsCarver c(nullptr);
+    carve_bs_index(c, n, Hkv, N, d);
+    return c.bytes();
+}
+size_t vs_prep_bytes(int n, int N, int kv) {
+    WsCarver c(nullptr);
+    carve_vs_prep(c, n, N, kv);
+    return c.bytes();
+}
+
+// Layer workspace: the VS and BS index outputs, then the scratch of each stage.
+struct LayerWs {
+    int32_t *v_idx, *s_idx, *blk_idx, *blk_cnt;
+    VsIndexWs vsi;
+    BsIndexWs bsi;
+    VsPrepWs prep;
+};
+LayerWs carve_layer(WsCarver& c, int nvs, int nbs, int Hkv, int N, int d, const mi_params& p) {
+    LayerWs w{};
+    const int nB = N / MI_BLOCK;
+    w.v_idx = c.take<int32_t>((size_t)nvs * p.vertical_size);
+    w.s_idx = c.take<int32_t>((size_t)nvs * p.slash_size);
+    w.blk_idx = c.take<int32_t>((size_t)nbs * nB * p.topk_blocks);
+    w.blk_cnt = c.take<int32_t>((size_t)nbs * nB);
+    if (nvs) w.vsi = carve_vs_index(c, nvs, N, p.last_q, true, true);
+    if (nbs) w.bsi = carve_bs_index(c, nbs, Hkv, N, d);
+    if (nvs) w.prep = carve_vs_prep(c, nvs, N, p.vertical_size);
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mi_status_str(int status) {
+    switch (status) {
+        case MI_OK: return "ok";
+        case MI_ERR_INVALID_ARG: return "invalid argument";
+        case MI_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+        case MI_ERR_WORKSPACE: return "workspace too small or misaligned";
+        case MI_ERR_CUDA: return "CUDA error (see mi_last_cuda_error)";
+        default: return "unknown status";
+    }
+}
+
+int mi_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* mi_version(void) { return "minfer 0.1 sm_100a"; }
+
+size_t mi_workspace_bytes(int op, int Hq, int Hkv, int N, int d, int n_heads, int last_q,
+                          int vertical_size, int slash_size, int topk_blocks) {
+    (void)topk_blocks;
+    if (Hq <= 0 || Hkv <= 0 || N <= 0 || N % MI_BLOCK || (d != 64 && d != 128)) return 0;
+    const int n = n_heads > 0 ? n_heads : Hq;
+    switch (op) {
+        case MI_OP_VS_INDEX:
+            if (last_q <= 0 || last_q > N) return 0;
+            return vs_index_bytes(n, N, last_q);
+        case MI_OP_BS_INDEX: return bs_index_bytes(n, Hkv, N, d);
+        case MI_OP_VS_ATTN: return vs_prep_bytes(n, N, vertical_size > 0 ? vertical_size : 1);
+        case MI_OP_BS_ATTN:
+        case MI_OP_ASHAPE_ATTN: return 256;
+        default: return 0;
+    }
+    (void)slash_size;
+}
+
+size_t mi_prefill_workspace_bytes(int Hq, int Hkv, int N, int d, const int8_t* pattern,
+                                  const mi_params* p) {
+    if (!p || Hq <= 0 || Hkv <= 0 || N <= 0 || N % MI_BLOCK || (d != 64 && d != 128)) return 0;
+    int nvs = 0, nbs = 0;
+    for (int h = 0; h < Hq; ++h) {
+        const int pt = pattern ? pattern[h] : -1;
+        if (pt == MI_PATTERN_VS || pt < 0) ++nvs;
+        if (pt == MI_PATTERN_BS || pt < 0) ++nbs;
+    }
+    WsCarver c(nullptr);
+    carve_layer(c, nvs, nbs, Hkv, N, d, *p);
+    return c.bytes();
+}
+
+int mi_vs_index(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d, float scale,
+                int last_q, int vertical_size, int slash_size, const int32_t* heads, int n_heads,
+                int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score, void* ws,
+                size_t ws_bytes, void* stream) {
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if ((rc = check_vs_params(N, last_q, vertical_size, slash_size))) return rc;
+    if ((vertical_size > 0 && !v_idx) || (slash_size > 0 && !s_idx)) return MI_ERR_INVALID_ARG;
+    const size_t need = vs_index_bytes(hl.n, N, last_q);
+    if ((rc = check_ws(ws, ws_bytes, need))) return rc;
+    if (hl.n == 0) return MI_OK;
+    WsCarver c(ws);
+    VsIndexWs w = carve_vs_index(c, hl.n, N, last_q, true, true);
+    set_pattern(hl, MI_PATTERN_VS);
+    return cuda_status(launch_vs_index(reinterpret_cast<const bf16*>(q),
+                                       reinterpret_cast<const bf16*>(k), Hq, Hkv, N, d,
+                                       eff_scale(scale, d), last_q, vertical_size, slash_size, hl,
+                                       v_idx, s_idx, v_score, s_score, w,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int mi_bs_index(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d, float scale,
+                int block, int topk, const int32_t* heads, int n_heads, int32_t* blk_idx,
+                int32_t* blk_cnt, void* ws, size_t ws_bytes, void* stream) {
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if (block != MI_BLOCK) return MI_ERR_UNSUPPORTED;
+    if (topk < 0) return MI_ERR_INVALID_ARG;
+    if (!blk_cnt || (topk > 0 && !blk_idx)) return MI_ERR_INVALID_ARG;
+    const size_t need = bs_index_bytes(hl.n, Hkv, N, d);
+    if ((rc = check_ws(ws, ws_bytes, need))) return rc;
+    if (hl.n == 0) return MI_OK;
+    WsCarver c(ws);
+    BsIndexWs w = carve_bs_index(c, hl.n, Hkv, N, d);
+    set_pattern(hl, MI_PATTERN_BS);
+    return cuda_status(launch_bs_index(reinterpret_cast<const bf16*>(q),
+                                       reinterpret_cast<const bf16*>(k), Hq, Hkv, N, d,
+                                       eff_scale(scale, d), topk, hl, blk_idx, blk_cnt, w,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+static void attn_common(AttnLaunch& a, const mi_bf16* q, const mi_bf16* k, const mi_bf16* v,
+                        int Hq, int Hkv, int N, int d, float scale, mi_bf16* out, float* lse,
+                        int32_t* err_count) {
+    memset(&a, 0, sizeof(a));
+    a.q = reinterpret_cast<const bf16*>(q);
+    a.k = reinterpret_cast<const bf16*>(k);
+    a.v = reinterpret_cast<const bf16*>(v);
+    a.out = reinterpret_cast<bf16*>(out);
+    a.lse = lse;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.N = N;
+    a.d = d;
+    a.scale = eff_scale(scale, d);
+    a.err_count = err_count;
+}
+
+int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                      int N, int d, float scale, const int32_t* v_idx, int vertical_size,
+                      const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
+                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                      void* stream) {
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if (!v || !out || vertical_size < 0 || slash_size < 0) return MI_ERR_INVALID_ARG;
+    if ((vertical_size > 0 && !v_idx) || (slash_size > 0 && !s_idx)) return MI_ERR_INVALID_ARG;
+    const int kv = vertical_size > 0 ? vertical_size : 1;
+    const size_t need = vs_prep_bytes(hl.n, N, kv);
+    if ((rc = check_ws(ws, ws_bytes, need))) return rc;
+    if (hl.n == 0) return MI_OK;
+    WsCarver c(ws);
+    VsPrepWs prep = carve_vs_prep(c, hl.n, N, kv);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = cuda_status(launch_vs_prep(v_idx, vertical_size, vertical_size, s_idx, slash_size,
+                                    slash_size, N, hl.n, prep, err_count, st));
+    if (rc) return rc;
+    AttnLaunch a;
+    attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
+    set_pattern(hl, MI_PATTERN_VS);
+    a.heads = hl;
+    a.dbits = prep.dbits;
+    a.vlist = prep.vlist;
+    a.vcnt = prep.vcnt;
+    a.vcap = prep.vcap;
+    return cuda_status(launch_sparse_attn(a, st));
+}
+
+int mi_block_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                         int N, int d, float scale, const int32_t* blk_idx,
+                         const int32_t* blk_cnt, int topk, int block, const int32_t* heads,
+                         int n_heads, mi_bf16* out, float* lse, int32_t* err_count, void* ws,
+                         size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if (block != MI_BLOCK) return MI_ERR_UNSUPPORTED;
+    if (!v || !out || topk < 0 || !blk_cnt || (topk > 0 && !blk_idx)) return MI_ERR_INVALID_ARG;
+    if (hl.n == 0) return MI_OK;
+    AttnLaunch a;
+    attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
+    set_pattern(hl, MI_PATTERN_BS);
+    a.heads = hl;
+    a.blk_idx = blk_idx;
+    a.blk_cnt = blk_cnt;
+    a.topk = topk;
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
+                   int d, float scale, int sink, int window, const int32_t* heads, int n_heads,
+                   mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                   void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if (!v || !out || sink < 0 || window < 1) return MI_ERR_INVALID_ARG;
+    if (hl.n == 0) return MI_OK;
+    AttnLaunch a;
+    attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
+    set_pattern(hl, MI_PATTERN_ASHAPE);
+    a.heads = hl;
+    a.sink = sink;
+    a.window = window;
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                     int N, int d, float scale, const int8_t* pattern, const mi_params* p,
+                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                     void* stream, void* const* stage_events) {
+    HeadList all;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, nullptr, 0, all);
+    if (rc) return rc;
+    if (!v || !out || !pattern || !p) return MI_ERR_INVALID_ARG;
+    HeadList vs{}, bs{};
+    int n_a = 0;
+    for (int h = 0; h < Hq; ++h) {
+        switch (pattern[h]) {
+            case MI_PATTERN_ASHAPE: all.e[h] = pack_head(h, MI_PATTERN_ASHAPE, n_a++); break;
+            case MI_PATTERN_VS:
+                all.e[h] = pack_head(h, MI_PATTERN_VS, vs.n);
+                vs.e[vs.n] = pack_head(h, MI_PATTERN_VS, vs.n);
+                ++vs.n;
+                break;
+            case MI_PATTERN_BS:
+                all.e[h] = pack_head(h, MI_PATTERN_BS, bs.n);
+                bs.e[bs.n] = pack_head(h, MI_PATTERN_BS, bs.n);
+                ++bs.n;
+                break;
+            default: return MI_ERR_INVALID_ARG;
+        }
+    }
+    if (vs.n && (rc = check_vs_params(N, p->last_q, p->vertical_size, p->slash_size))) return rc;
+    if (bs.n && p->topk_blocks < 0) return MI_ERR_INVALID_ARG;
+    if (n_a && (p->sink < 0 || p->window < 1)) return MI_ERR_INVALID_ARG;
+    mi_params pp = *p;
+    if (!vs.n) pp.vertical_size = pp.slash_size = 0;
+    if (!bs.n) pp.topk_blocks = 0;
+    if (vs.n && pp.vertical_size < 1) pp.vertical_size = 1;  // keep carved buffers non-empty
+    WsCarver sizer(nullptr);
+    carve_layer(sizer, vs.n, bs.n, Hkv, N, d, pp);
+    if ((rc = check_ws(ws, ws_bytes, sizer.bytes()))) return rc;
+
+    WsCarver c(ws);
+    LayerWs w = carve_layer(c, vs.n, bs.n, Hkv, N, d, pp);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const double sc = eff_scale(scale, d);
+    auto rec = [&](int i) -> int {
+        if (!stage_events || !stage_events[i]) return MI_OK;
+        return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st));
+    };
+    if ((rc = rec(MI_STAGE_START))) return rc;
+    const bf16* qb = reinterpret_cast<const bf16*>(q);
+    const bf16* kb = reinterpret_cast<const bf16*>(k);
+    if (vs.n) {
+        rc = cuda_status(launch_vs_index(qb, kb, Hq, Hkv, N, d, sc, pp.last_q, pp.vertical_size,
+                                         pp.slash_size, vs, w.v_idx, w.s_idx, nullptr, nullptr,
+                                         w.vsi, st));
+        if (rc) return rc;
+    }
+    if (bs.n) {
+        rc = cuda_status(launch_bs_index(qb, kb, Hq, Hkv, N, d, sc, pp.topk_blocks, bs, w.blk_idx,
+                                         w.blk_cnt, w.bsi, st));
+        if (rc) return rc;
+    }
+    if ((rc = rec(MI_STAGE_INDEX_DONE))) return rc;
+    if (vs.n) {
+        rc = cuda_status(launch_vs_prep(w.v_idx, pp.vertical_size, pp.vertical_size, w.s_idx,
+                                        pp.slash_size, pp.slash_size, N, vs.n, w.prep, err_count,
+                                        st));
+        if (rc) return rc;
+    }
+    AttnLaunch a;
+    attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
+    a.heads = all;
+    a.dbits = w.prep.dbits;
+    a.vlist = w.prep.vlist;
+    a.vcnt = w.prep.vcnt;
+    a.vcap = w.prep.vcap;
+    a.blk_idx = w.blk_idx;
+    a.blk_cnt = w.blk_cnt;
+    a.topk = pp.topk_blocks;
+    a.sink = pp.sink;
+    a.window = pp.window;
+    if ((rc = cuda_status(launch_sparse_attn(a, st)))) return rc;
+    return rec(MI_STAGE_ATTN_DONE);
+}
+
+}  // extern "C"

@@ -1,0 +1,879 @@
+// attn.cu -- dynamic sparse attention on B200 tensor cores (tcgen05 + TMEM,
+// operands staged by TMA), one engine for all three MInference patterns.
+//
+// MInference 1.0 (aifetchly guide, "Technical Deep Dive"): each head runs
+// causal flash-style attention with an online softmax over only its selected
+// keys: the sink plus local band (A-shape), the chosen 64x64 blocks
+// (Block-Sparse), or the gathered vertical columns plus the 64x64 tiles its
+// slash diagonals touch (Vertical-Slash), without counting a key twice.
+//
+// Work item = one query head x one 256-row "super tile" (four 64-row query
+// blocks).  The CTA holds the super tile as two 128-row slots that share
+// every key group brought into shared memory:
+//   warps 0-3  softmax, slot 0 (TMEM lanes 0-127 = rows 0-127)
+//   warps 4-7  softmax, slot 1 (rows 128-255)
+//   warp 8     producer: enumerates the key groups of the item and loads
+//              them (TMA for pairs of 64-key blocks, cp.async gathers for
+//              vertical columns), two stages deep
+//   warp 9     MMA issuer: S = Q K^T (SS form) and O += P V (TS form, P read
+//              from TMEM), FA-style ping-pong between the two slots.
+// A key group is 128 keys: two (not necessarily adjacent) 64-key blocks, or
+// up to 128 gathered columns.  Each block / column carries a 4-bit mask, one
+// bit per query block, so one group serves rows with different masks; rows
+// whose bit is clear see -inf.  Only the diagonal block of a row, the edges
+// of an A-shape band and gathered columns need element-level tests.
+//
+// TMEM (512 columns): slot x uses S at [256x, 256x+128) (P, bf16 pairs,
+// aliases its first 64 columns) and O at [256x+128, 256x+128+d).
+#include <cfloat>
+#include <cstring>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace minfer {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kGroupKeys = 128;
+constexpr int kPanelBytes = 128 * 128;  // 128 rows x one 64-column (128-byte) panel
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by >8
+
+enum : int { kGrpNone = 0, kGrpTiles = 1, kGrpGather = 2 };
+
+struct GroupDesc {
+    int type, last, need, ncols;
+    int b0, b1, m0, m1;
+    int cols[kGroupKeys];
+    uint8_t cm[kGroupKeys];
+};
+
+struct GatherHeld {
+    int cols[kGroupKeys];
+    uint8_t cm[kGroupKeys];
+};
+
+// Sequence number of the last launch in which a CTA gave up waiting; later
+// CTAs of that launch exit at once instead of timing out one by one.
+__device__ unsigned int g_abort_seq = 0;
+
+struct AttnParams {
+    unsigned int seq;  // launch sequence number (never 0)
+    const bf16* k;
+    const bf16* v;
+    bf16* out;
+    float* lse;
+    int Hq, Hkv, N, nB, n_super;
+    float scale_log2;
+    const uint32_t* dbits;
+    int nBw;
+    const int32_t* vlist;
+    const int32_t* vcnt;
+    int vcap;
+    const int32_t* blk_idx;
+    const int32_t* blk_cnt;
+    int topk;
+    int sink, window;
+    int32_t* err;
+    HeadList heads;
+};
+
+template <int D>
+struct Layout {
+    static constexpr int kQBytes = 128 * D * 2;   // one slot of Q
+    static constexpr int kKVBytes = kGroupKeys * D * 2;
+    static constexpr int q_off = 0;
+    static constexpr int k_off = q_off + 2 * kQBytes;
+    static constexpr int v_off = k_off + 2 * kKVBytes;
+    static constexpr int desc_off = v_off + 2 * kKVBytes;
+    static constexpr int held_off = desc_off + 2 * (int)sizeof(GroupDesc);
+    static constexpr int bar_off = (held_off + (int)sizeof(GatherHeld) + 15) & ~15;
+    static constexpr int kNumBars = 12;
+    static constexpr int misc_off = bar_off + kNumBars * 8;
+    static constexpr int patmap_off = misc_off + 16;
+    static size_t bytes(int patmap_words) {
+        size_t b = (size_t)patmap_off + (size_t)patmap_words * 4 + 1024;  // +1024: base alignment
+        // d = 64 is small enough for two CTAs per SM, but TMEM holds one: ask for enough
+        // shared memory that the SM schedules one at a time.
+        return b < 120 * 1024 ? 120 * 1024 : b;
+    }
+};
+
+struct Bars {
+    uint64_t* q_full;
+    uint64_t* kv_full;   // [2]
+    uint64_t* kv_empty;  // [2]
+    uint64_t* s_full;    // [2]
+    uint64_t* p_full;    // [2]
+    uint64_t* o_done;    // [2]
+    uint64_t* drain;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void set_abort(volatile int* abort, int32_t* err, unsigned int seq) {
+    *abort = 1;
+    if (err) atomicOr(err, 1 << 30);
+    atomicExch(&g_abort_seq, seq);
+}
+
+// ------------------------------------------------------------- producer
+template <int D>
+struct Producer {
+    using L = Layout<D>;
+    const AttnParams& p;
+    const CUtensorMap* tmK;
+    const CUtensorMap* tmV;
+    uint8_t* sm;
+    Bars bars;
+    volatile int* abort;
+    GroupDesc* desc;
+    GatherHeld* held;
+    int g;       // KV head
+    int pub = 0; // groups published
+    int lane;
+    bool ok = true;
+
+    __device__ bool acquire(int& s) {
+        s = pub & 1;
+        if (pub >= 2) {
+            bool w = true;
+            if (lane == 0) w = mbar_wait(&bars.kv_empty[s], ((pub >> 1) - 1) & 1, abort);
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) {
+                if (lane == 0) set_abort(abort, p.err, p.seq);
+                ok = false;
+                return false;
+            }
+        }
+        return true;
+    }
+
+    __device__ void tiles(int b0, int m0, int b1, int m1) {
+        if (!ok) return;
+        int s;
+        if (!acquire(s)) return;
+        if (lane == 0) {
+            GroupDesc& d = desc[s];
+            d.type = kGrpTiles;
+            d.last = 0;
+            d.need = (((m0 | m1) & 0x3) ? 1 : 0) | (((m0 | m1) & 0xC) ? 2 : 0);
+            d.ncols = 0;
+            d.b0 = b0;
+            d.b1 = b1;
+            d.m0 = m0;
+            d.m1 = m1;
+            mbar_arrive_expect_tx(&bars.kv_full[s], 2 * L::kKVBytes);
+            uint8_t* kd = sm + L::k_off + s * L::kKVBytes;
+            uint8_t* vd = sm + L::v_off + s * L::kKVBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = g * p.N + 64 * (h ? b1 : b0);
+#pragma unroll
+                for (int pn = 0; pn < D / 64; ++pn) {
+                    tma_load_2d(kd + pn * kPanelBytes + h * (kPanelBytes / 2), tmK, 64 * pn, row,
+                                &bars.kv_full[s]);
+                    tma_load_2d(vd + pn * kPanelBytes + h * (kPanelBytes / 2), tmV, 64 * pn, row,
+                                &bars.kv_full[s]);
+                }
+            }
+        }
+        __syncwarp();
+        ++pub;
+    }
+
+    __device__ void gather(int n) {
+        if (!ok) return;
+        int s;
+        if (!acquire(s)) return;
+        GroupDesc& d = desc[s];
+        int need = 0;
+        for (int c = lane; c < kGroupKeys; c += 32) {
+            const bool v = c < n;
+            const int col = v ? held->cols[c] : held->cols[0];
+            const int cm = v ? held->cm[c] : 0;
+            d.cols[c] = col;
+            d.cm[c] = (uint8_t)cm;
+            need |= cm;
+        }
+        for (int off = 16; off >= 1; off >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, off);
+        if (lane == 0) {
+            d.type = kGrpGather;
+            d.last = 0;
+            d.need = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
+            d.ncols = n;
+            d.b0 = d.b1 = -1;
+            d.m0 = d.m1 = 0;
+        }
+        __syncwarp();
+        uint8_t* kd = sm + L::k_off + s * L::kKVBytes;
+        uint8_t* vd = sm + L::v_off + s * L::kKVBytes;
+        constexpr int kChunks = D / 8;  // 16-byte chunks per row
+        const bf16* kb = p.k + (size_t)g * p.N * D;
+        const bf16* vb = p.v + (size_t)g * p.N * D;
+        for (int idx = lane; idx < kGroupKeys * kChunks; idx += 32) {
+            const int r = idx / kChunks, c = idx % kChunks;
+            const size_t src = (size_t)d.cols[r] * D + c * 8;
+            const int dst = (c >> 3) * kPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+            cp_async_16(kd + dst, kb + src);
+            cp_async_16(vd + dst, vb + src);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.kv_full[s]);
+        ++pub;
+    }
+
+    __device__ void finish() {
+        if (!ok) return;
+        int s;
+        if (!acquire(s)) return;
+        if (lane == 0) {
+            GroupDesc& d = desc[s];
+            d.type = kGrpNone;
+            d.last = 1;
+            d.need = 0;
+            d.ncols = 0;
+            mbar_arrive(&bars.kv_full[s]);
+        }
+        __syncwarp();
+        ++pub;
+    }
+
+    // Wait (bounded) until every copy this warp started has landed, so that
+    // no TMA write can reach shared memory after the CTA exits.
+    __device__ void drain() {
+        if (lane != 0) return;
+        for (int u = pub - 2; u < pub; ++u) {
+            if (u < 0) continue;
+            mbar_wait_budget(&bars.kv_full[u & 1], (u >> 1) & 1);
+        }
+    }
+};
+
+__device__ __forceinline__ bool bit_of(const uint32_t* bits, int i) {
+    return (bits[i >> 5] >> (i & 31)) & 1u;
+}
+
+template <int D>
+__device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                             const CUtensorMap* tmV, uint8_t* sm, const Bars& bars,
+                             volatile int* abort, uint32_t* patmap, int pos, int T) {
+    using L = Layout<D>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t e = p.heads.e[pos];
+    const int qh = head_qh(e), pattern = head_pattern(e), pidx = head_pidx(e);
+    const int g = kv_head_of(qh, p.Hq, p.Hkv);
+    const int qb0 = 4 * T;
+    const int nqb = min(4, p.nB - qb0);
+    const int bmax = min(qb0 + 3, p.nB - 1);
+
+    if (lane == 0) {
+        prefetch_tmap(tmQ);
+        prefetch_tmap(tmK);
+        prefetch_tmap(tmV);
+        mbar_arrive_expect_tx(bars.q_full, 2 * L::kQBytes);
+        for (int x = 0; x < 2; ++x)
+            for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_2d(sm + L::q_off + x * L::kQBytes + pn * kPanelBytes, tmQ, 64 * pn,
+                            qh * p.N + 256 * T + 128 * x, bars.q_full);
+    }
+
+    // per-pattern block map
+    if (pattern == MI_PATTERN_VS) {
+        const uint32_t* src = p.dbits + (size_t)pidx * p.nBw;
+        for (int w = lane; w < p.nBw; w += 32) patmap[w] = src[w];
+    } else if (pattern == MI_PATTERN_BS) {
+        const int nwords = (bmax + 8) / 8;  // 8 nibbles per word
+        for (int w = lane; w < nwords; w += 32) patmap[w] = 0;
+        __syncwarp();
+        for (int qq = 0; qq < nqb; ++qq) {
+            const int qb = qb0 + qq;
+            const int cnt = min(p.blk_cnt[(size_t)pidx * p.nB + qb], p.topk);
+            const int32_t* lst = p.blk_idx + ((size_t)pidx * p.nB + qb) * p.topk;
+            for (int t = lane; t < cnt; t += 32) {
+                const int bk = lst[t];
+                if (bk == -1) continue;  // padding
+                if (bk < 0 || bk > qb) {
+                    if (p.err) atomicAdd(p.err, 1);
+                    continue;
+                }
+                atomicOr(&patmap[bk >> 3], (1u << qq) << ((bk & 7) * 4));
+            }
+        }
+    }
+    __syncwarp();
+
+    Producer<D> pr{p, tmK, tmV, sm, bars, abort,
+                   reinterpret_cast<GroupDesc*>(sm + L::desc_off),
+                   reinterpret_cast<GatherHeld*>(sm + L::held_off), g};
+    pr.lane = lane;
+
+    // --- 64-key blocks, ascending, paired into 128-key groups
+    int pend_b = -1, pend_m = 0;
+    for (int base = 0; base <= bmax && pr.ok; base += 32) {
+        const int b = base + lane;
+        int m = 0;
+        if (b <= bmax) {
+            if (pattern == MI_PATTERN_VS) {
+                for (int qq = 0; qq < nqb; ++qq) {
+                    const int delta = qb0 + qq - b;
+                    if (delta >= 0 && bit_of(patmap, delta)) m |= 1 << qq;
+                }
+            } else if (pattern == MI_PATTERN_BS) {
+                m = (patmap[b >> 3] >> ((b & 7) * 4)) & 0xF;
+            } else {
+                for (int qq = 0; qq < nqb; ++qq) {
+                    const int qb = qb0 + qq;
+                    if (b <= qb && (64 * b < p.sink || 64 * (qb - b) - 63 < p.window))
+                        m |= 1 << qq;
+                }
+            }
+        }
+        unsigned bal = __ballot_sync(0xffffffffu, m != 0);
+        while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const int mm = __shfl_sync(0xffffffffu, m, src);
+            if (pend_b < 0) {
+                pend_b = base + src;
+                pend_m = mm;
+            } else {
+                pr.tiles(pend_b, pend_m, base + src, mm);
+                pend_b = -1;
+            }
+        }
+    }
+    if (pend_b >= 0) pr.tiles(pend_b, pend_m, pend_b, 0);
+
+    // --- Vertical-Slash: gathered columns not already inside a computed tile
+    if (pattern == MI_PATTERN_VS && pr.ok) {
+        const int vc = p.vcnt[pidx];
+        const int32_t* vl = p.vlist + (size_t)pidx * p.vcap;
+        const long long rlast = min(256LL * T + 255, (long long)p.N - 1);
+        GatherHeld* held = pr.held;
+        int n_held = 0;
+        for (int base = 0; base < vc && pr.ok; base += 32) {
+            const int t = base + lane;
+            const int j = t < vc ? vl[t] : 0x7fffffff;
+            int m = 0;
+            if (j <= rlast) {
+                for (int qq = 0; qq < nqb; ++qq) {
+                    const int qb = qb0 + qq;
+                    if (j < 64 * (qb + 1)) {
+                        const int delta = qb - (j >> 6);
+                        if (!bit_of(patmap, delta)) m |= 1 << qq;
+                    }
+                }
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, m != 0);
+            const int rank = __popc(bal & ((1u << lane) - 1u));
+            const int navail = __popc(bal);
+            const int take = min(navail, kGroupKeys - n_held);
+            if (m && rank < take) {
+                held->cols[n_held + rank] = j;
+                held->cm[n_held + rank] = (uint8_t)m;
+            }
+            __syncwarp();
+            n_held += take;
+            if (n_held == kGroupKeys) {
+                pr.gather(n_held);
+                n_held = 0;
+                if (m && rank >= take) {
+                    held->cols[rank - take] = j;
+                    held->cm[rank - take] = (uint8_t)m;
+                }
+                __syncwarp();
+                n_held = navail - take;
+            }
+            if (__any_sync(0xffffffffu, j > rlast)) break;  // the list is sorted
+        }
+        if (n_held > 0) pr.gather(n_held);
+    }
+    pr.finish();
+
+    // make sure Q and every started load have landed before the CTA can exit
+    if (lane == 0) mbar_wait_budget(bars.q_full, 0);
+    pr.drain();
+}
+
+// ------------------------------------------------------------- MMA issuer
+template <int D>
+__device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int32_t* err,
+                        unsigned int seq, uint32_t tmem) {
+    using L = Layout<D>;
+    const uint32_t idS = idesc_bf16_f32(128, kGroupKeys, false);
+    const uint32_t idO = idesc_bf16_f32(128, D, true);
+    const uint32_t q_addr = smem_u32(sm + L::q_off);
+    const uint32_t k_addr = smem_u32(sm + L::k_off);
+    const uint32_t v_addr = smem_u32(sm + L::v_off);
+    const GroupDesc* desc = reinterpret_cast<const GroupDesc*>(sm + L::desc_off);
+
+    int pend[2] = {-1, -1}, pend_stage[2] = {0, 0}, npv[2] = {0, 0}, np[2] = {0, 0};
+    int uses[2] = {0, 0};
+    bool ok = mbar_wait(bars.q_full, 0, abort);
+    int g = 0;
+    while (ok) {
+        const int s = g & 1;
+        if (!mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        const int type = desc[s].type, need = desc[s].need, last = desc[s].last;
+        if (type == kGrpNone)
+            mbar_arrive(&bars.kv_empty[s]);
+        else
+            uses[s] = __popc(need);
+        for (int x = 0; x < 2 && ok; ++x) {
+            if (pend[x] >= 0) {
+                if (!mbar_wait(&bars.p_full[x], np[x] & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                ++np[x];
+                tc_fence_after();
+                const int st = pend_stage[x];
+                const uint32_t tP = tmem + 256 * x;
+                const uint32_t tO = tmem + 256 * x + 128;
+#pragma unroll
+                for (int kk = 0; kk < kGroupKeys / 16; ++kk) {
+                    const uint64_t bdesc =
+                        sw128_desc(v_addr + st * L::kKVBytes + kk * 2048, kPanelBytes, 1024);
+                    mma_ts(tO, tP + kk * 8, bdesc, idO, (npv[x] > 0 || kk > 0) ? 1u : 0u);
+                }
+                ++npv[x];
+                if (--uses[st] == 0) mma_commit(&bars.kv_empty[st]);
+                pend[x] = -1;
+            }
+            if (type != kGrpNone && ((need >> x) & 1)) {
+                const uint32_t tS = tmem + 256 * x;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int pn = kk >> 2, off = (kk & 3) * 32;
+                    const uint64_t adesc =
+                        sw128_desc(q_addr + x * L::kQBytes + pn * kPanelBytes + off, 16, 1024);
+                    const uint64_t bdesc =
+                        sw128_desc(k_addr + s * L::kKVBytes + pn * kPanelBytes + off, 16, 1024);
+                    mma_ss(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars.s_full[x]);
+                pend[x] = g;
+                pend_stage[x] = s;
+            }
+        }
+        if (!ok || last) break;
+        ++g;
+    }
+    if (!ok) set_abort(abort, err, seq);
+    for (int x = 0; x < 2; ++x)
+        if (npv[x] > 0) mma_commit(&bars.o_done[x]);
+    // every MMA must have finished before TMEM is released
+    mma_commit(bars.drain);
+    mbar_wait_budget(bars.drain, 0);
+}
+
+// ------------------------------------------------------------- softmax
+template <int D>
+__device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
+                            volatile int* abort, uint32_t tmem, int pos, int T) {
+    using L = Layout<D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int x = warp >> 2, lg = warp & 3;
+    const int t = lg * 32 + lane;         // row within the slot = TMEM lane
+    const int rloc = 128 * x + t;         // row within the super tile
+    const int qi = rloc >> 6;             // query block within the super tile
+    const long long i = 256LL * T + rloc; // global row
+    const uint32_t e = p.heads.e[pos];
+    const int qh = head_qh(e), pattern = head_pattern(e);
+    const bool ashape = pattern == MI_PATTERN_ASHAPE;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    const uint32_t tS = tmem + 256 * x + lane_off;
+    const uint32_t tO = tmem + 256 * x + 128 + lane_off;
+    const GroupDesc* desc = reinterpret_cast<const GroupDesc*>(sm + L::desc_off);
+
+    float m = -INFINITY, l = 0.f;
+    int ns = 0;
+    bool ok = true;
+    for (int g = 0;; ++g) {
+        const int s = g & 1;
+        if (!mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort)) {
+            ok = false;
+            break;
+        }
+        const GroupDesc& d = desc[s];
+        const int type = d.type, last = d.last;
+        if (type != kGrpNone && ((d.need >> x) & 1)) {
+            if (!mbar_wait(&bars.s_full[x], ns & 1, abort)) {
+                ok = false;
+                break;
+            }
+            ++ns;
+            tc_fence_after();
+            float v[kGroupKeys];
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    tmem_ld32(tS + 32 * c, r);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) v[32 * c + u] = __uint_as_float(r[u]) * p.scale_log2;
+                }
+            }
+            if (type == kGrpTiles) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int b = h ? d.b1 : d.b0;
+                    const int bit = ((h ? d.m1 : d.m0) >> qi) & 1;
+                    const long long j0 = 64LL * b;
+                    const bool full = bit && (j0 + 63 <= i) &&
+                                      (!ashape || j0 + 63 < p.sink || i - j0 < p.window);
+                    if (!full) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c) {
+                            const long long j = j0 + c;
+                            const bool keep = bit && j <= i &&
+                                              (!ashape || j < p.sink || i - j < p.window);
+                            if (!keep) v[64 * h + c] = -INFINITY;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kGroupKeys; ++c) {
+                    const bool keep = ((d.cm[c] >> qi) & 1) && (long long)d.cols[c] <= i;
+                    if (!keep) v[c] = -INFINITY;
+                }
+            }
+            float mx = v[0];
+#pragma unroll
+            for (int c = 1; c < kGroupKeys; ++c) mx = fmaxf(mx, v[c]);
+            if (mx > m + kRescaleThreshold) {
+                const float alpha = ex2(m - mx);  // 0 while m is -inf
+                if (ns > 1) {
+                    uint32_t o[32];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        tmem_ld32(tO + 32 * c, o);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+                        tmem_st32(tO + 32 * c, o);
+                    }
+                }
+                l *= alpha;
+                m = mx;
+            }
+            const float mu = (m == -INFINITY) ? 0.f : m;
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const float p0 = ex2(v[64 * c + 2 * u] - mu);
+                    const float p1 = ex2(v[64 * c + 2 * u + 1] - mu);
+                    rs += p0 + p1;
+                    pk[u] = pack_bf16(p0, p1);
+                }
+                tmem_st32(tS + 32 * c, pk);
+            }
+            l += rs;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars.p_full[x]);
+        }
+        mbar_arrive(&bars.kv_empty[s]);
+        if (last) break;
+    }
+
+    // epilogue: O / l -> bf16, lse
+    bool have = ns > 0 && ok;
+    if (have) have = mbar_wait(&bars.o_done[x], 0, abort);
+    if (!ok || (ns > 0 && !have)) set_abort(abort, p.err, p.seq);
+    tc_fence_after();
+    const bool row_ok = i < p.N;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    bf16* orow = p.out + ((size_t)qh * p.N + (size_t)(row_ok ? i : 0)) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (have) {
+            tmem_ld32(tO + 32 * c, o);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            pk[u] = pack_bf16(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
+        if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+    }
+    if (row_ok && p.lse)
+        p.lse[(size_t)qh * p.N + i] =
+            l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+    tc_fence_before();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ AttnParams p) {
+    using L = Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    // 128-byte swizzled operands need a 1024-byte aligned base
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::bar_off);
+    Bars bars{bar + 0, bar + 1, bar + 3, bar + 5, bar + 7, bar + 9, bar + 11};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::misc_off);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::misc_off + 4);
+    uint32_t* patmap = reinterpret_cast<uint32_t*>(sm + L::patmap_off);
+
+    if (*reinterpret_cast<volatile unsigned int*>(&g_abort_seq) == p.seq) return;
+    const int n = p.heads.n;
+    const int T = p.n_super - 1 - (int)(blockIdx.x / n);  // longest (latest) tiles first
+    const int pos = (int)(blockIdx.x % n);
+    const int warp = threadIdx.x >> 5;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars.q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars.kv_full[s], 1);
+            mbar_init(&bars.kv_empty[s], 1 + kSoftmaxThreads);
+            mbar_init(&bars.s_full[s], 1);
+            mbar_init(&bars.p_full[s], 128);
+            mbar_init(&bars.o_done[s], 1);
+        }
+        mbar_init(bars.drain, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 8) {
+        run_softmax<D>(p, sm, bars, abort, tmem, pos, T);
+    } else if (warp == kProducerWarp) {
+        run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
+    } else {
+        if ((threadIdx.x & 31) == 0) run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
+        __syncwarp();
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------- VS prep
+// Per VS head: slash offsets -> block-diagonal bitmap D (offset o touches
+// deltas o/64 and, unless o % 64 == 0, o/64 + 1), vertical columns -> sorted
+// unique list.  Entries outside [0, N) other than the -1 padding are counted.
+__global__ void __launch_bounds__(1024) vs_prep_kernel(const int32_t* __restrict__ v_idx,
+                                                       int kv_stride, int kv,
+                                                       const int32_t* __restrict__ s_idx,
+                                                       int ks_stride, int ks, int N,
+                                                       VsPrepWs ws, int32_t* err) {
+    extern __shared__ uint32_t dsm[];
+    __shared__ int warp_tot[33];
+    const int pos = blockIdx.x;
+    const int nB = N / 64, nBw = (nB + 31) / 32, nW = N / 32;
+    uint32_t* col = ws.colbits + (size_t)pos * nW;
+    for (int w = threadIdx.x; w < nBw; w += blockDim.x) dsm[w] = 0;
+    for (int w = threadIdx.x; w < nW; w += blockDim.x) col[w] = 0;
+    __syncthreads();
+    for (int t = threadIdx.x; t < ks; t += blockDim.x) {
+        const int o = s_idx[(size_t)pos * ks_stride + t];
+        if (o < 0 || o >= N) {
+            if (o != -1 && err) atomicAdd(err, 1);
+            continue;
+        }
+        const int a = o >> 6;
+        atomicOr(&dsm[a >> 5], 1u << (a & 31));
+        if ((o & 63) && a + 1 < nB) atomicOr(&dsm[(a + 1) >> 5], 1u << ((a + 1) & 31));
+    }
+    for (int t = threadIdx.x; t < kv; t += blockDim.x) {
+        const int j = v_idx[(size_t)pos * kv_stride + t];
+        if (j < 0 || j >= N) {
+            if (j != -1 && err) atomicAdd(err, 1);
+            continue;
+        }
+        atomicOr(&col[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < nBw; w += blockDim.x) ws.dbits[(size_t)pos * nBw + w] = dsm[w];
+    // ordered compaction of the column bitmap
+    int32_t* out = ws.vlist + (size_t)pos * ws.vcap;
+    int base_out = 0;
+    for (int base = 0; base < nW; base += blockDim.x) {
+        const int w = base + threadIdx.x;
+        const uint32_t bits = w < nW ? col[w] : 0u;
+        const int c = __popc(bits);
+        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+        int incl = c;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) warp_tot[wp] = incl;
+        __syncthreads();
+        if (wp == 0) {
+            const int tv = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+            int ti = tv;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, ti, off);
+                if (lane >= off) ti += y;
+            }
+            warp_tot[lane] = ti - tv;
+            if (lane == 31) warp_tot[32] = ti;
+        }
+        __syncthreads();
+        int o = base_out + warp_tot[wp] + incl - c;
+        uint32_t b = bits;
+        while (b) {
+            const int k = __ffs(b) - 1;
+            b &= b - 1;
+            if (o < ws.vcap) out[o] = w * 32 + k;
+            ++o;
+        }
+        base_out += warp_tot[32];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) ws.vcnt[pos] = min(base_out, ws.vcap);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over [rows][d] bf16, 64-column x box_rows boxes, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
+    using L = Layout<D>;
+    CUtensorMap tmQ, tmK, tmV;
+    if (!make_map(&tmQ, a.q, (long long)a.Hq * a.N, D, 128) ||
+        !make_map(&tmK, a.k, (long long)a.Hkv * a.N, D, 64) ||
+        !make_map(&tmV, a.v, (long long)a.Hkv * a.N, D, 64))
+        return cudaErrorInvalidValue;
+    static unsigned int seq = 0;
+    AttnParams p;
+    memset(&p, 0, sizeof(p));
+    if (++seq == 0) ++seq;
+    p.seq = seq;
+    p.k = a.k;
+    p.v = a.v;
+    p.out = a.out;
+    p.lse = a.lse;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.N = a.N;
+    p.nB = a.N / 64;
+    p.n_super = (a.N + 255) / 256;
+    p.scale_log2 = (float)(a.scale * 1.4426950408889634);
+    p.dbits = a.dbits;
+    p.nBw = (p.nB + 31) / 32;
+    p.vlist = a.vlist;
+    p.vcnt = a.vcnt;
+    p.vcap = a.vcap;
+    p.blk_idx = a.blk_idx;
+    p.blk_cnt = a.blk_cnt;
+    p.topk = a.topk;
+    p.sink = a.sink;
+    p.window = a.window;
+    p.err = a.err_count;
+    p.heads = a.heads;
+    const int patmap_words = p.nBw > p.nB / 8 + 1 ? p.nBw : p.nB / 8 + 1;
+    const size_t smem = L::bytes(patmap_words);
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(a.heads.n * p.n_super);
+    sparse_attn_kernel<D><<<grid, kThreads, smem, st>>>(tmQ, tmK, tmV, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv) {
+    VsPrepWs w{};
+    const int nB = N / 64, nBw = (nB + 31) / 32;
+    w.vcap = kv < N ? kv : N;
+    if (w.vcap < 1) w.vcap = 1;
+    w.dbits = c.take<uint32_t>((size_t)n_heads * nBw);
+    w.colbits = c.take<uint32_t>((size_t)n_heads * (N / 32));
+    w.vlist = c.take<int32_t>((size_t)n_heads * w.vcap);
+    w.vcnt = c.take<int32_t>((size_t)n_heads);
+    return w;
+}
+
+cudaError_t launch_vs_prep(const int32_t* v_idx, int kv_stride, int kv, const int32_t* s_idx,
+                           int ks_stride, int ks, int N, int n_heads, const VsPrepWs& ws,
+                           int32_t* err_count, cudaStream_t st) {
+    if (n_heads == 0) return cudaSuccess;
+    const int nBw = (N / 64 + 31) / 32;
+    vs_prep_kernel<<<n_heads, 1024, nBw * sizeof(uint32_t), st>>>(v_idx, kv_stride, kv, s_idx,
+                                                                  ks_stride, ks, N, ws, err_count);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st) {
+    if (a.heads.n == 0) return cudaSuccess;
+    return a.d == 128 ? launch_attn_d<128>(a, st) : launch_attn_d<64>(a, st);
+}
+
+}  // namespace minfer

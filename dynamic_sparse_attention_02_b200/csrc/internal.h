@@ -1,0 +1,111 @@
+// internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/minfer.h"
+
+namespace minfer {
+
+using bf16 = __nv_bfloat16;
+
+// Query heads of one launch, in list order.  Each entry packs
+// qh (bits 0-11), pattern (bits 12-13) and the head's position in the
+// per-pattern index arrays (bits 16-31).
+struct HeadList {
+    int n;
+    uint32_t e[MI_MAX_HEADS];
+};
+
+__host__ __device__ inline uint32_t pack_head(int qh, int pattern, int pidx) {
+    return (uint32_t)qh | ((uint32_t)pattern << 12) | ((uint32_t)pidx << 16);
+}
+__host__ __device__ inline int head_qh(uint32_t e) { return (int)(e & 0xFFFu); }
+__host__ __device__ inline int head_pattern(uint32_t e) { return (int)((e >> 12) & 0x3u); }
+__host__ __device__ inline int head_pidx(uint32_t e) { return (int)(e >> 16); }
+// grouped-query attention, contiguous groups
+__host__ __device__ inline int kv_head_of(int qh, int Hq, int Hkv) {
+    return (int)(((long long)qh * Hkv) / Hq);
+}
+
+// Bump allocator over the caller's workspace.  With base == nullptr it only
+// measures, so size queries and launches carve identically.
+struct WsCarver {
+    char* base;
+    size_t off = 0;
+    explicit WsCarver(void* b) : base(static_cast<char*>(b)) {}
+    template <class T>
+    T* take(size_t count) {
+        off = (off + 255) & ~size_t(255);
+        T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+        off += count * sizeof(T);
+        return p;
+    }
+    size_t bytes() const { return (off + 255) & ~size_t(255); }
+};
+
+// ----------------------------------------------------------- VS index
+constexpr int kVsChunk = 1024;  // keys per CTA in the score passes
+
+struct VsIndexWs {
+    double* m_part;  // [n_heads][L][nchunks]
+    double* l_part;
+    float* vscore;   // [n_heads][N]
+    float* sscore;   // [n_heads][N]
+};
+VsIndexWs carve_vs_index(WsCarver& c, int n_heads, int N, int L, bool need_vscore,
+                         bool need_sscore);
+cudaError_t launch_vs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
+                            double scale, int L, int kv, int ks, const HeadList& heads,
+                            int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
+                            const VsIndexWs& ws, cudaStream_t st);
+
+// ----------------------------------------------------------- BS index
+struct BsIndexWs {
+    float* qm;  // [n_heads][nB][d]
+    float* km;  // [Hkv][nB][d]
+};
+BsIndexWs carve_bs_index(WsCarver& c, int n_heads, int Hkv, int N, int d);
+cudaError_t launch_bs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
+                            double scale, int topk, const HeadList& heads, int32_t* blk_idx,
+                            int32_t* blk_cnt, const BsIndexWs& ws, cudaStream_t st);
+
+// ----------------------------------------------------------- attention
+struct VsPrepWs {
+    uint32_t* dbits;    // [n_heads][nBw]   slash diagonals -> block-diagonal set
+    uint32_t* colbits;  // [n_heads][N/32]  vertical columns as a bitmap
+    int32_t* vlist;     // [n_heads][vcap]  sorted unique columns
+    int32_t* vcnt;      // [n_heads]
+    int vcap;
+};
+VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv);
+cudaError_t launch_vs_prep(const int32_t* v_idx, int kv_stride, int kv, const int32_t* s_idx,
+                           int ks_stride, int ks, int N, int n_heads, const VsPrepWs& ws,
+                           int32_t* err_count, cudaStream_t st);
+
+struct AttnLaunch {
+    const bf16 *q, *k, *v;
+    bf16* out;
+    float* lse;
+    int Hq, Hkv, N, d;
+    double scale;
+    HeadList heads;  // pattern + per-pattern position per entry
+    // Vertical-Slash
+    const uint32_t* dbits;
+    const int32_t* vlist;
+    const int32_t* vcnt;
+    int vcap;
+    // Block-Sparse
+    const int32_t* blk_idx;
+    const int32_t* blk_cnt;
+    int topk;
+    // A-shape
+    int sink, window;
+    int32_t* err_count;
+};
+cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);
+
+}  // namespace minfer

@@ -1,0 +1,118 @@
+// topk.cuh -- block-wide top-k by radix select, ties broken toward the lower
+// index, result written in ascending index order.
+//
+// Keys are fp32 scores mapped to order-preserving uint32 (larger score ->
+// larger key).  Four 8-bit histogram passes find the k-th largest key T and
+// how many of the keys equal to T are still needed; one ordered compaction
+// pass then keeps every key > T and the first `need_eq` keys == T.
+#pragma once
+
+#include <cstdint>
+
+namespace minfer {
+
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+    uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Block-wide exclusive prefix sum of one int per thread (blockDim.x a
+// multiple of 32, <= 1024).  `warp_tot` holds 33 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? warp_tot[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += y;
+        }
+        if (lane < nwarps) warp_tot[lane] = wi - w;  // exclusive per warp
+        if (lane == 31) warp_tot[32] = wi;
+    }
+    __syncthreads();
+    const int res = warp_tot[warp] + incl - v;
+    total = warp_tot[32];
+    __syncthreads();
+    return res;
+}
+
+// Shared scratch for one block-wide selection.
+struct TopkSmem {
+    uint32_t hist[256];
+    int warp_tot[33];
+    uint32_t prefix;
+    int remaining;
+};
+
+// Find threshold key T and the number of keys equal to T to keep, for the
+// top k (1 <= k < n) of keys get(0..n-1).
+template <class Get>
+__device__ void block_radix_select(const Get& get, int n, int k, TopkSmem& s, uint32_t& thr,
+                                   int& need_eq) {
+    if (threadIdx.x == 0) {
+        s.prefix = 0;
+        s.remaining = k;
+    }
+    uint32_t mask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = threadIdx.x; b < 256; b += blockDim.x) s.hist[b] = 0;
+        __syncthreads();
+        const uint32_t prefix = s.prefix;
+        for (int j = threadIdx.x; j < n; j += blockDim.x) {
+            const uint32_t key = get(j);
+            if ((key & mask) == prefix) atomicAdd(&s.hist[(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int rem = s.remaining;
+            int b = 255;
+            for (; b > 0; --b) {
+                const int c = (int)s.hist[b];
+                if (c >= rem) break;
+                rem -= c;
+            }
+            s.remaining = rem;
+            s.prefix = prefix | ((uint32_t)b << shift);
+        }
+        __syncthreads();
+        mask |= 255u << shift;
+    }
+    thr = s.prefix;
+    need_eq = s.remaining;
+    __syncthreads();
+}
+
+// Write the selected indices in ascending order to out[0..k).
+template <class Get>
+__device__ void block_select_compact(const Get& get, int n, int k, uint32_t thr, int need_eq,
+                                     TopkSmem& s, int32_t* out) {
+    int eq_base = 0, sel_base = 0;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        uint32_t key = 0;
+        if (j < n) key = get(j);
+        const int gt = (j < n && key > thr) ? 1 : 0;
+        const int eq = (j < n && key == thr) ? 1 : 0;
+        int eq_tot;
+        const int eq_rank = eq_base + block_exclusive_scan(eq, s.warp_tot, eq_tot);
+        const int sel = gt | (eq & (eq_rank < need_eq ? 1 : 0));
+        int sel_tot;
+        const int pos = sel_base + block_exclusive_scan(sel, s.warp_tot, sel_tot);
+        if (sel && pos < k) out[pos] = j;
+        eq_base += eq_tot;
+        sel_base += sel_tot;
+    }
+}
+
+}  // namespace minfer

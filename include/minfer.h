@@ -1,0 +1,212 @@
+/*
+ * minfer.h -- C ABI of libminfer.so: MInference dynamic sparse attention
+ * prefill (MInference 1.0, arXiv 2407.02490) on NVIDIA B200 (sm_100a).
+ *
+ * The method (MInference 1.0 abstract; hotpaper.ai summary "key idea";
+ * aifetchly "MInference 1.0 Guide", "The Three Fundamental Attention
+ * Topologies" and "Technical Deep Dive") has two stages per attention head:
+ *   1. an online sparse index: Vertical-Slash (VS) heads score every key
+ *      column and every diagonal from the last `last_q` queries and keep the
+ *      top ones; Block-Sparse (BS) heads score 64-token mean-pooled query and
+ *      key blocks and keep the top key blocks per query block;
+ *   2. causal softmax attention computed only over the selected columns and
+ *      diagonals, blocks, or (A-shape heads) sink tokens plus a local window.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - q is [Hq][N][d], k and v are [Hkv][N][d], out is [Hq][N][d]: contiguous
+ *    row-major bf16 (mi_bf16 = raw bf16 bits) in DEVICE memory owned by the
+ *    caller.  Query head h reads KV head floor(h * Hkv / Hq) (grouped-query
+ *    attention, contiguous groups).
+ *  - Supported shapes: d in {64, 128}; N a multiple of 64 with N >= 64;
+ *    Hq a multiple of Hkv; 1 <= Hq <= MI_MAX_HEADS.  Others return
+ *    MI_ERR_UNSUPPORTED (shape) or MI_ERR_INVALID_ARG (inconsistent).
+ *  - `heads` is a HOST array of `n_heads` query-head ids (each processed at
+ *    most once); NULL means all Hq heads in order.  Per-head index arrays
+ *    (v_idx, s_idx, blk_idx, blk_cnt, scores) are indexed by POSITION in that
+ *    list; out / lse are indexed by absolute head.  Heads not listed are not
+ *    touched.
+ *  - `scale` is the softmax scale; pass 0 for the default 1/sqrt(d).
+ *  - `ws` / `ws_bytes`: caller-owned device workspace, at least the size
+ *    mi_workspace_bytes() returns for the same arguments, 256-byte aligned.
+ *    The library allocates no memory of any kind.
+ *  - `stream` is a cudaStream_t (as void*); all work is enqueued on it,
+ *    asynchronously.  No entry point synchronises the device or the stream
+ *    or copies device data to the host.
+ *  - Every entry point validates its arguments on the host first.  On any
+ *    error nothing is launched and the status says why; MI_ERR_CUDA keeps the
+ *    cudaError_t in thread-local storage (mi_last_cuda_error()).
+ *  - `err_count` (optional, device int32, may be NULL): the attention entry
+ *    points add the number of index entries they skipped (out of range) to
+ *    it; if a device-side wait ever gives up (a bounded wait, never expected
+ *    in a correct run) bit 30 is set in it.
+ *  - Budgets larger than the candidate count are clamped (vertical_size and
+ *    slash_size to N, topk to the number of causal blocks): "budgets that
+ *    cover everything" give dense causal attention.
+ */
+#ifndef MINFER_H
+#define MINFER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mi_bf16; /* raw bf16 bit pattern */
+
+enum {
+    MI_OK = 0,
+    MI_ERR_INVALID_ARG = 1, /* null pointer, negative size, Hq % Hkv != 0, bad head id */
+    MI_ERR_UNSUPPORTED = 2, /* d not in {64,128}, N % 64 != 0, N < last_q, too many heads */
+    MI_ERR_WORKSPACE = 3,   /* ws too small or misaligned */
+    MI_ERR_CUDA = 4         /* a CUDA call failed; see mi_last_cuda_error() */
+};
+
+enum { MI_PATTERN_ASHAPE = 0, MI_PATTERN_VS = 1, MI_PATTERN_BS = 2 };
+
+enum {
+    MI_OP_VS_INDEX = 1,
+    MI_OP_BS_INDEX = 2,
+    MI_OP_VS_ATTN = 3,
+    MI_OP_BS_ATTN = 4,
+    MI_OP_ASHAPE_ATTN = 5
+};
+
+#define MI_MAX_HEADS 256
+#define MI_BLOCK 64
+
+/* Per-pattern parameters of one layer (all heads of a pattern share them). */
+typedef struct {
+    int last_q;        /* VS: number of final queries that score columns/diagonals */
+    int vertical_size; /* VS: columns kept per head */
+    int slash_size;    /* VS: diagonals kept per head */
+    int topk_blocks;   /* BS: key blocks kept per 64-row query block */
+    int sink;          /* A-shape: keys 0..sink-1 always kept */
+    int window;        /* A-shape: keys i-window+1 .. i kept for row i */
+} mi_params;
+
+/* Stage boundaries recorded by mi_prefill_layer when stage_events != NULL. */
+enum { MI_STAGE_START = 0, MI_STAGE_INDEX_DONE = 1, MI_STAGE_ATTN_DONE = 2, MI_STAGE_EVENTS = 3 };
+
+/* Static description of a status code; never NULL. */
+const char* mi_status_str(int status);
+
+/* cudaError_t of the last MI_ERR_CUDA returned on this thread (0 if none). */
+int mi_last_cuda_error(void);
+
+/* Library version, e.g. "minfer 0.1 sm_100a". */
+const char* mi_version(void);
+
+/*
+ * Workspace bytes for one call of `op` with these shapes (n_heads <= 0 means
+ * all Hq heads).  Arguments the op does not use are ignored.  Returns 0 for
+ * arguments the op would reject.
+ */
+size_t mi_workspace_bytes(int op, int Hq, int Hkv, int N, int d, int n_heads, int last_q,
+                          int vertical_size, int slash_size, int topk_blocks);
+
+/*
+ * Workspace bytes for mi_prefill_layer.  `pattern` is the host pattern table
+ * [Hq] (NULL: budget for any table).
+ */
+size_t mi_prefill_workspace_bytes(int Hq, int Hkv, int N, int d, const int8_t* pattern,
+                                  const mi_params* p);
+
+/*
+ * Vertical-Slash index (hotpaper.ai "key idea"; guide "2. The Vertical-Slash
+ * Pattern").  For each listed head h and each of the last L = last_q rows
+ * i = N-L .. N-1: row softmax of scale * q_i . k_j over j <= i; vertical[j]
+ * sums the probabilities of column j over the L rows, slash[o] sums those of
+ * diagonal o = i - j.  Scores are computed in fp64 and ranked as fp32.
+ * The top vertical_size columns and top slash_size diagonals (ties: lower
+ * index first) are written sorted ascending:
+ *   v_idx [n_heads][vertical_size], s_idx [n_heads][slash_size] (int32,
+ *   device); entries past min(budget, N) are set to -1.
+ *   v_score, s_score [n_heads][N] fp32 (device, optional): the scores.
+ * Requires 1 <= last_q <= N.
+ */
+int mi_vs_index(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d, float scale,
+                int last_q, int vertical_size, int slash_size, const int32_t* heads, int n_heads,
+                int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score, void* ws,
+                size_t ws_bytes, void* stream);
+
+/*
+ * Block-Sparse index (hotpaper.ai "key idea": 64-token mean pooling; guide
+ * "Block-Sparse Kernel Mechanics": block score against the mean key of each
+ * block, keep the top-k).  Qm[b] / Km[b] are means of 64 rows; for query
+ * block bq the candidates are key blocks bk <= bq with score
+ * scale * Qm[bq] . Km[bk] (fp64 sums of fp32 means).  The top
+ * min(topk, bq+1) (ties: lower block first) are written sorted ascending:
+ *   blk_idx [n_heads][N/64][topk] int32 (device; unused entries -1),
+ *   blk_cnt [n_heads][N/64] int32 (device).
+ * `block` must be 64.
+ */
+int mi_bs_index(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d, float scale,
+                int block, int topk, const int32_t* heads, int n_heads, int32_t* blk_idx,
+                int32_t* blk_cnt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Vertical-Slash sparse attention (guide, "Vertical-Slash Kernel
+ * Mechanics": online softmax over the gathered columns and the diagonals).
+ * Row i attends key j <= i iff j is one of the head's vertical columns, or
+ * the 64x64 tile holding (i, j) is touched by one of its slash diagonals
+ * (diagonal o touches the tiles with block-diagonal delta = bq - bk,
+ * |o - 64 delta| <= 63; such tiles are computed whole, causally masked).
+ * A key is never counted twice.  v_idx [n_heads][vertical_size] and
+ * s_idx [n_heads][slash_size] (device int32) may be unsorted and may repeat
+ * entries; entries outside [0, N) are skipped (counted in err_count).
+ * out [Hq][N][d] bf16; lse [Hq][N] fp32 natural-log sum of exp (optional).
+ * A row with no allowed key gets out = 0 and lse = -inf.
+ */
+int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                      int N, int d, float scale, const int32_t* v_idx, int vertical_size,
+                      const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
+                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Block-sparse attention (guide, "3. The Block-Sparse Pattern": only the
+ * selected 64x64 tiles are computed).  Row i of query block bq = i / 64
+ * attends key j <= i iff j / 64 is among the first blk_cnt[bq] entries of
+ * blk_idx[bq] (device int32, layouts as produced by mi_bs_index; entries may
+ * be unsorted or repeated; entries outside [0, bq] are skipped and counted).
+ * `block` must be 64.  out / lse as for mi_vs_sparse_attn.
+ */
+int mi_block_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                         int N, int d, float scale, const int32_t* blk_idx,
+                         const int32_t* blk_cnt, int topk, int block, const int32_t* heads,
+                         int n_heads, mi_bf16* out, float* lse, int32_t* err_count, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/*
+ * A-shape attention (guide, "1. The A-Shape Pattern": attention sinks plus a
+ * local causal band).  Row i attends key j <= i iff j < sink or
+ * i - j < window (the window counts the query itself).  sink >= 0,
+ * window >= 1.  out / lse as for mi_vs_sparse_attn.
+ */
+int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
+                   int d, float scale, int sink, int window, const int32_t* heads, int n_heads,
+                   mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/*
+ * One attention layer with a per-head pattern table (guide, "Phase 2: The
+ * Online Dynamic Kernel Router"): `pattern` is a HOST int8 [Hq] of
+ * MI_PATTERN_* codes.  Builds the VS and BS indices for the heads that need
+ * them, then runs one sparse-attention launch over all heads, each with its
+ * own pattern; all on `stream`, no host-device synchronisation.
+ * stage_events (optional): MI_STAGE_EVENTS cudaEvent_t handles (as void*),
+ * recorded on `stream` at the stage boundaries.
+ */
+int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                     int N, int d, float scale, const int8_t* pattern, const mi_params* p,
+                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                     void* stream, void* const* stage_events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MINFER_H */

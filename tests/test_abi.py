@@ -1,0 +1,132 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host with the documented status
+(on this GPU-less machine any launch would fail with MI_ERR_CUDA instead, so
+getting the validation code shows nothing was launched)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from dynamic_sparse_attention_02_b200 import binding as B
+from dynamic_sparse_attention_02_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "minfer.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(mi_\w+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) == 11
+    assert sorted(B.EXPORTS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert B.mi_status_str(code)
+    assert B.mi_status_str(99) == "unknown status"
+    assert "sm_100a" in B.mi_version()
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation runs first
+
+
+def vs_index(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, Hq=4, Hkv=2, N=512, d=128, scale=0.0, last_q=64, kv=16, ks=32,
+             heads=None, n_heads=0, v_idx=FAKE, s_idx=FAKE, vs=None, ss=None, ws=FAKE,
+             ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return lib.mi_vs_index(a["q"], a["k"], a["Hq"], a["Hkv"], a["N"], a["d"], a["scale"],
+                           a["last_q"], a["kv"], a["ks"], a["heads"], a["n_heads"], a["v_idx"],
+                           a["s_idx"], a["vs"], a["ss"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_vs_index_validation(lib):
+    assert vs_index(lib, q=None) == B.MI_ERR_INVALID_ARG
+    assert vs_index(lib, Hq=3) == B.MI_ERR_INVALID_ARG              # Hq % Hkv
+    assert vs_index(lib, d=96) == B.MI_ERR_UNSUPPORTED
+    assert vs_index(lib, N=500) == B.MI_ERR_UNSUPPORTED             # N % 64
+    assert vs_index(lib, last_q=1024 + 64, N=4096) == B.MI_ERR_UNSUPPORTED
+    assert vs_index(lib, last_q=1024) == B.MI_ERR_UNSUPPORTED       # last_q > N
+    assert vs_index(lib, last_q=0) == B.MI_ERR_INVALID_ARG
+    assert vs_index(lib, kv=-1) == B.MI_ERR_INVALID_ARG
+    assert vs_index(lib, v_idx=None) == B.MI_ERR_INVALID_ARG
+    assert vs_index(lib, ws_bytes=16) == B.MI_ERR_WORKSPACE
+    assert vs_index(lib, ws=ctypes.c_void_p(0x1001)) == B.MI_ERR_WORKSPACE  # misaligned
+    dup = (ctypes.c_int32 * 2)(1, 1)
+    assert vs_index(lib, heads=dup, n_heads=2) == B.MI_ERR_INVALID_ARG
+    bad = (ctypes.c_int32 * 1)(4)
+    assert vs_index(lib, heads=bad, n_heads=1) == B.MI_ERR_INVALID_ARG
+    assert vs_index(lib, Hq=512, Hkv=2) == B.MI_ERR_UNSUPPORTED     # > MI_MAX_HEADS
+
+
+def test_attention_validation(lib):
+    f = FAKE
+    # block-sparse: block must be 64, topk >= 0
+    assert lib.mi_block_sparse_attn(f, f, f, 4, 2, 512, 128, 0.0, f, f, 8, 32, None, 0, f, None,
+                                    None, None, 0, None) == B.MI_ERR_UNSUPPORTED
+    assert lib.mi_block_sparse_attn(f, f, f, 4, 2, 512, 128, 0.0, f, f, -1, 64, None, 0, f, None,
+                                    None, None, 0, None) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_block_sparse_attn(f, f, None, 4, 2, 512, 128, 0.0, f, f, 8, 64, None, 0, f,
+                                    None, None, None, 0, None) == B.MI_ERR_INVALID_ARG
+    # A-shape: window >= 1, sink >= 0
+    assert lib.mi_ashape_attn(f, f, f, 4, 2, 512, 128, 0.0, 64, 0, None, 0, f, None, None, None,
+                              0, None) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_ashape_attn(f, f, f, 4, 2, 512, 128, 0.0, -1, 8, None, 0, f, None, None, None,
+                              0, None) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_ashape_attn(f, f, f, 4, 2, 520, 128, 0.0, 4, 8, None, 0, f, None, None, None,
+                              0, None) == B.MI_ERR_UNSUPPORTED
+    # VS attention: workspace
+    assert lib.mi_vs_sparse_attn(f, f, f, 4, 2, 512, 128, 0.0, f, 8, f, 8, None, 0, f, None,
+                                 None, f, 8, None) == B.MI_ERR_WORKSPACE
+    # BS index
+    assert lib.mi_bs_index(f, f, 4, 2, 512, 128, 0.0, 32, 8, None, 0, f, f, f, 1 << 30,
+                           None) == B.MI_ERR_UNSUPPORTED
+
+
+def test_prefill_layer_validation(lib):
+    f = FAKE
+    p = B.make_params()
+    bad = np.array([0, 1, 2, 7], np.int8)
+    assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, bad.ctypes.data_as(ctypes.c_void_p),
+                                ctypes.byref(p), f, None, None, f, 1 << 30, None,
+                                None) == B.MI_ERR_INVALID_ARG
+    good = np.array([0, 1, 2, 1], np.int8)
+    assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, good.ctypes.data_as(ctypes.c_void_p),
+                                ctypes.byref(p), f, None, None, f, 16, None,
+                                None) == B.MI_ERR_WORKSPACE
+    assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, None, ctypes.byref(p), f, None,
+                                None, f, 1 << 30, None, None) == B.MI_ERR_INVALID_ARG
+    p2 = B.make_params(last_q=1024)
+    assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, good.ctypes.data_as(ctypes.c_void_p),
+                                ctypes.byref(p2), f, None, None, f, 1 << 30, None,
+                                None) == B.MI_ERR_UNSUPPORTED
+
+
+def test_workspace_queries(lib):
+    a = B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, 131072, 128, 32, 64, 1000, 6096)
+    b = B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, 131072, 128, 4, 64, 1000, 6096)
+    assert a > b > 0 and a % 256 == 0
+    assert B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, 131072, 128, 32, 200000) == 0
+    assert B.mi_workspace_bytes(B.MI_OP_BS_INDEX, 32, 8, 131072, 128) > 0
+    assert B.mi_workspace_bytes(B.MI_OP_VS_ATTN, 32, 8, 131072, 128, 0, 0, 1000) > 0
+    assert B.mi_workspace_bytes(99, 32, 8, 131072, 128) == 0
+    p = B.make_params()
+    full = B.mi_prefill_workspace_bytes(32, 8, 131072, 128, None, p)
+    vs_only = B.mi_prefill_workspace_bytes(32, 8, 131072, 128, np.ones(32, np.int8), p)
+    a_only = B.mi_prefill_workspace_bytes(32, 8, 131072, 128, np.zeros(32, np.int8), p)
+    assert full >= vs_only > a_only >= 0
