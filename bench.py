@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark: one MInference dynamic-sparse prefill layer per step on B200.
+
+A step is one pass of the whole hot path over one layer of synthetic input:
+mi_prefill_layer = per-head index estimation + slash/vertical prep + one
+sparse-attention launch.  Default workload: the LLaMA-3-8B-shaped 128K layer
+(32 query heads, 8 KV heads, d = 128, N = 131072, every head Vertical-Slash
+with last_q = 64, vertical 1000, slash 6096).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl minfer|reference]
+
+Multi-GPU runs (torchrun, one process per GPU) are independent replicas: the
+layer does not shard, so there is no data-path collective; the step time is
+the max over ranks and the reported ms/layer is that time divided by the
+number of layers all ranks processed.
+
+--impl reference times the CPU oracle (the only reference implementation of
+this method here) on a bounded sample of the same workload, extrapolated to
+the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_sparse_attention_02_b200 import synth  # noqa: E402
+
+METRIC = "sparse prefill attn ms/layer (index+attn) at 128K/1M; tensor-pipe util %"
+UNIT = "ms/layer"
+_T0 = time.time()
+
+
+def log(msg):
+    """Progress on stderr (the JSON result goes to stdout)."""
+    print(f"[bench {time.time() - _T0:7.1f}s] {msg}", file=sys.stderr, flush=True)
+
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SOURCES = ["attn.cu", "ptx.cuh", "internal.h"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="minfer", choices=["minfer", "reference"])
+    ap.add_argument("--workload", default="vs_n128k_llama3_8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0,
+                    help="approximate CPU seconds for the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def params_of(w, B):
+    return B.make_params(last_q=w.last_q, vertical_size=w.vertical_size, slash_size=w.slash_size,
+                         topk_blocks=w.topk_blocks, sink=w.sink, window=w.window)
+
+
+def attn_source_sha():
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "dynamic_sparse_attention_02_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per attention launch from a committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    entry = rec.get(workload)
+    if not entry or entry.get("source_sha") != attn_source_sha():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def vs_useful_flops(v_idx, s_idx, N, d):
+    """Useful FLOPs of one VS head: 4*d per (row, key) pair over computed 64x64
+    tiles (slash diagonals -> block diagonals D) plus 64 rows per gathered
+    column per query block (columns outside D tiles).  Returns (flops, tiles,
+    gathered column-blocks)."""
+    nB = N // 64
+    s = s_idx[(s_idx >= 0) & (s_idx < N)]
+    D = np.zeros(nB + 1, bool)
+    a = s // 64
+    D[a] = True
+    D[np.minimum(a + 1, nB)[(s % 64) != 0]] = True
+    D = D[:nB]
+    deltas = np.nonzero(D)[0]
+    tiles = int(np.sum(nB - deltas))
+    V = np.unique(v_idx[(v_idx >= 0) & (v_idx < N)])
+    cnt_le = np.cumsum(D)  # |{delta in D : delta <= x}|
+    bj = V // 64
+    cols = int(np.sum((nB - bj) - cnt_le[nB - 1 - bj]))
+    return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
+
+
+# ----------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, x, n_rows, rng, heads=(0,)):
+    """Time the CPU oracle on a bounded sample; returns (extrapolated ms/layer, desc, cores)."""
+    import oracle
+    pattern = x["pattern"]
+    t_index = 0.0
+    t_rows = 0.0
+    rows_done = 0
+    for h in heads:
+        g = h * w.Hkv // w.Hq
+        qs = x["q"][h:h + 1].float().cpu()
+        ks = x["k"][g:g + 1].float().cpu()
+        vs = x["v"][g:g + 1].float().cpu()
+        rows = np.sort(rng.choice(w.N, size=n_rows, replace=False))
+        pt = int(pattern[h])
+        t0 = time.perf_counter()
+        if pt == synth.PATTERN_VS:
+            vi, si, _, _ = oracle.vs_index(qs, ks, 0, w.last_q, w.vertical_size, w.slash_size)
+        elif pt == synth.PATTERN_BS:
+            bi, bc = oracle.bs_index(qs, ks, 0, w.topk_blocks)
+        t1 = time.perf_counter()
+        if pt == synth.PATTERN_VS:
+            oracle.attn_vs(qs, ks, vs, 0, vi, si, rows=rows)
+        elif pt == synth.PATTERN_BS:
+            oracle.attn_bs(qs, ks, vs, 0, bi, bc, rows=rows)
+        else:
+            oracle.attn_ashape(qs, ks, vs, 0, w.sink, w.window, rows=rows)
+        t2 = time.perf_counter()
+        t_index += t1 - t0
+        t_rows += t2 - t1
+        rows_done += n_rows
+    nh = len(heads)
+    ms = 1e3 * (t_index / nh * w.Hq + t_rows / rows_done * w.N * w.Hq)
+    desc = (f"index of {nh} head(s) + {n_rows} seeded random rows of attention per head at "
+            f"N={w.N}, extrapolated to {w.Hq} heads x {w.N} rows")
+    return ms, desc, oracle.num_threads()
+
+
+def rows_for_budget(w, budget_s):
+    # ~4*d*N/2 flops per row in fp64 loops at ~1 GFLOP/s per core, plus the index
+    import oracle
+    cores = max(1, oracle.num_threads())
+    per_row = 4.0 * w.d * w.N / 2 / (1.0e9 * cores)
+    return int(min(2048, max(16, budget_s * 0.6 / max(per_row, 1e-9))))
+
+
+# ----------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.workload(args.workload)
+    x = synth.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    rng = np.random.default_rng(w.seed)
+    total = args.steps + args.warmup
+    n_rows = max(16, rows_for_budget(w, 150.0 / max(total, 1)) // 2)
+    for _ in range(args.warmup):
+        oracle_sample(w, x, n_rows, rng)
+    vals = []
+    desc, cores = "", 1
+    for _ in range(args.steps):
+        ms, desc, cores = oracle_sample(w, x, n_rows, rng)
+        vals.append(ms)
+    v = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": v,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "pattern": w.pattern, "last_q": w.last_q, "vertical_size": w.vertical_size,
+            "slash_size": w.slash_size, "topk_blocks": w.topk_blocks, "sink": w.sink,
+            "window": w.window, "parallelism": "replicas",
+            "l2": "inputs larger than L2 (q 1 GiB, k+v 512 MiB at 128K); no flush"}
+
+
+def run_minfer(args):
+    from dynamic_sparse_attention_02_b200 import binding as B
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(val):
+        if dist is None:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = synth.workload(args.workload)
+    log(f"generating {w.name}")
+    x = synth.make_inputs(w, device=str(dev))
+    torch.cuda.synchronize()
+    q, k, v = x["q"], x["k"], x["v"]
+    pattern = x["pattern"]
+    params = params_of(w, B)
+    ws = torch.empty(B.mi_prefill_workspace_bytes(w.Hq, w.Hkv, w.N, w.d, pattern, params),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    n_vs = int(np.sum(pattern == synth.PATTERN_VS))
+    n_bs = int(np.sum(pattern == synth.PATTERN_BS))
+    launches_per_step = (4 + 1 if n_vs else 0) + (3 if n_bs else 0) + 1
+
+    def step(ev):
+        B.mi_prefill_layer(q, k, v, pattern, params, out=out, ws=ws, stage_events=ev)
+
+    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
+    for i in range(args.warmup):
+        step(warm_ev)
+        torch.cuda.synchronize()
+        log(f"warmup step {i}: index {warm_ev[0].elapsed_time(warm_ev[1]):.2f} ms, "
+            f"attn {warm_ev[2].elapsed_time(warm_ev[3]):.2f} ms")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
+           for _ in range(args.steps)]
+    for e in evs:
+        for ee in e:
+            ee.record()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_step = t_start.elapsed_time(t_end) / args.steps
+    ms_index = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    ms_prep = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms_attn = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    ms_step_max = max_over_ranks(ms_step)
+    log(f"timed {args.steps} steps: {ms_step:.2f} ms/step (attn {ms_attn:.2f} ms)")
+
+    # end to end through the public API: host inputs in, host output back
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        n_e2e = max(1, min(args.steps, 5))
+
+        def step_e2e():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            B.mi_prefill_layer(dq, dk, dv, pattern, params, out=out, ws=ws)
+            hout.copy_(out, non_blocking=True)
+
+        step_e2e()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n_e2e):
+            step_e2e()
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e)
+        log(f"e2e {ms_e2e:.2f} ms/step")
+        e2e = {"value": ms_e2e / world, "unit": UNIT,
+               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+               "d2h_bytes_per_step": int(hout.numel() * 2), "steps": n_e2e}
+        assert torch.equal(hout, out.cpu()), "e2e output differs from the device output"
+
+    # algorithmic work of the attention launch (from this layer's own index)
+    useful = 0.0
+    tiles = 0
+    cols = 0
+    if n_vs == w.Hq:
+        v_idx, s_idx = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size)
+        vi, si = v_idx.cpu().numpy(), s_idx.cpu().numpy()
+        for h in range(w.Hq):
+            f, t, c = vs_useful_flops(vi[h], si[h], w.N, w.d)
+            useful += f
+            tiles += t
+            cols += c
+    dense_eq = 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = useful / (ms_attn * 1e-3) / 1e12 if useful else None
+    traffic = recorded_traffic(w.name)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rng = np.random.default_rng(w.seed)
+            n_rows = rows_for_budget(w, args.cpu_budget_s)
+            log(f"oracle baseline: {n_rows} rows")
+            ms_cpu, desc, cores = oracle_sample(w, x, n_rows, rng)
+            log("oracle baseline done")
+            cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": desc}
+        line = {
+            "metric": METRIC, "value": ms_step_max / world, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step_max,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w),
+            "ms_index": ms_index, "ms_prep": ms_prep, "ms_attn": ms_attn,
+            "tile_density": (tiles / (w.Hq * (w.N // 64) * (w.N // 64 + 1) / 2)) if tiles else None,
+            "gathered_column_blocks": cols,
+            "eff_tflops": achieved,
+            "dense_eq_tflops": dense_eq / (ms_step_max * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": (achieved / peak) if achieved else None,
+                         "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                         "traffic": traffic,
+                         "flops_per_launch": useful},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_minfer(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

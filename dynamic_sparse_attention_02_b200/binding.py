@@ -22,14 +22,15 @@ LIB_PATH = os.path.join(HERE, "libminfer.so")
 MI_OK, MI_ERR_INVALID_ARG, MI_ERR_UNSUPPORTED, MI_ERR_WORKSPACE, MI_ERR_CUDA = range(5)
 MI_PATTERN_ASHAPE, MI_PATTERN_VS, MI_PATTERN_BS = 0, 1, 2
 MI_OP_VS_INDEX, MI_OP_BS_INDEX, MI_OP_VS_ATTN, MI_OP_BS_ATTN, MI_OP_ASHAPE_ATTN = 1, 2, 3, 4, 5
-MI_STAGE_START, MI_STAGE_INDEX_DONE, MI_STAGE_ATTN_DONE, MI_STAGE_EVENTS = 0, 1, 2, 3
+MI_STAGE_START, MI_STAGE_INDEX_DONE, MI_STAGE_PREP_DONE, MI_STAGE_ATTN_DONE, MI_STAGE_EVENTS = (
+    0, 1, 2, 3, 4)
 MI_MAX_HEADS = 256
 MI_BLOCK = 64
 
 # every symbol include/minfer.h declares
 EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
-           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer"]
+           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure"]
 
 
 class MinferError(RuntimeError):
@@ -75,6 +76,7 @@ def _lib_handle():
         lib.mi_ashape_attn.argtypes = [P, P, P, I, I, I, I, F, I, I, P, I, P, P, P, P, SZ, P]
         lib.mi_prefill_layer.argtypes = [P, P, P, I, I, I, I, F, P, ctypes.POINTER(mi_params),
                                          P, P, P, P, SZ, P, P]
+        lib.mi_debug_wait_failure.argtypes = [P]
         for name in EXPORTS[5:]:
             getattr(lib, name).restype = I
         _lib = lib
@@ -119,6 +121,14 @@ def _workspace(nbytes, device, ws):
             raise ValueError("workspace too small")
         return ws
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def mi_debug_wait_failure():
+    """First device wait that gave up since the last read (all zeros if none); clears it."""
+    rec = (ctypes.c_int32 * 8)()
+    _check("mi_debug_wait_failure", _lib_handle().mi_debug_wait_failure(rec))
+    keys = ["seq", "site", "block", "thread", "group", "parity", "r6", "r7"]
+    return dict(zip(keys, list(rec)))
 
 
 def mi_status_str(status: int) -> str:

@@ -355,6 +355,7 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
                                         st));
         if (rc) return rc;
     }
+    if ((rc = rec(MI_STAGE_PREP_DONE))) return rc;
     AttnLaunch a;
     attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
     a.heads = all;
@@ -369,6 +370,15 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
     a.window = pp.window;
     if ((rc = cuda_status(launch_sparse_attn(a, st)))) return rc;
     return rec(MI_STAGE_ATTN_DONE);
+}
+
+int mi_debug_wait_failure(int32_t* record8) {
+    if (!record8) return MI_ERR_INVALID_ARG;
+    int rec[8];
+    const int rc = cuda_status(read_wait_failure(rec));
+    if (rc) return rc;
+    for (int i = 0; i < 8; ++i) record8[i] = rec[i];
+    return MI_OK;
 }
 
 }  // extern "C"

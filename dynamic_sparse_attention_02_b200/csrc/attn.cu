@@ -63,6 +63,31 @@ struct GatherHeld {
 // CTAs of that launch exit at once instead of timing out one by one.
 __device__ unsigned int g_abort_seq = 0;
 
+// First wait that gave up since the record was last read:
+// {launch seq, site, block, thread, group, parity, 0, 0}; site 0 = none.
+__device__ int g_wait_fail[8];
+
+enum : int {
+    kSiteProducerEmpty = 1,
+    kSiteMmaQ = 2,
+    kSiteMmaFull = 3,
+    kSiteMmaP = 4,
+    kSiteSoftmaxFull = 5,
+    kSiteSoftmaxS = 6,
+    kSiteSoftmaxO = 7
+};
+
+__device__ void record_wait_failure(unsigned int seq, int site, int group, int parity) {
+    if (atomicCAS(&g_wait_fail[1], 0, site) == 0) {
+        g_wait_fail[0] = (int)seq;
+        g_wait_fail[2] = (int)blockIdx.x;
+        g_wait_fail[3] = (int)threadIdx.x;
+        g_wait_fail[4] = group;
+        g_wait_fail[5] = parity;
+        __threadfence();
+    }
+}
+
 struct AttnParams {
     unsigned int seq;  // launch sequence number (never 0)
     const bf16* k;
@@ -156,7 +181,10 @@ struct Producer {
             if (lane == 0) w = mbar_wait(&bars.kv_empty[s], ((pub >> 1) - 1) & 1, abort);
             w = __shfl_sync(0xffffffffu, w, 0);
             if (!w) {
-                if (lane == 0) set_abort(abort, p.err, p.seq);
+                if (lane == 0) {
+                    if (!*abort) record_wait_failure(p.seq, kSiteProducerEmpty, pub, ((pub >> 1) - 1) & 1);
+                    set_abort(abort, p.err, p.seq);
+                }
                 ok = false;
                 return false;
             }
@@ -428,10 +456,12 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
     int pend[2] = {-1, -1}, pend_stage[2] = {0, 0}, npv[2] = {0, 0}, np[2] = {0, 0};
     int uses[2] = {0, 0};
     bool ok = mbar_wait(bars.q_full, 0, abort);
+    if (!ok && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, 0);
     int g = 0;
     while (ok) {
         const int s = g & 1;
         if (!mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort)) {
+            if (!*abort) record_wait_failure(seq, kSiteMmaFull, g, (g >> 1) & 1);
             ok = false;
             break;
         }
@@ -444,6 +474,7 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
         for (int x = 0; x < 2 && ok; ++x) {
             if (pend[x] >= 0) {
                 if (!mbar_wait(&bars.p_full[x], np[x] & 1, abort)) {
+                    if (!*abort) record_wait_failure(seq, kSiteMmaP, g, np[x] & 1);
                     ok = false;
                     break;
                 }
@@ -513,14 +544,16 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     bool ok = true;
     for (int g = 0;; ++g) {
         const int s = g & 1;
-        if (!mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort))) {
+            if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxFull, g, (g >> 1) & 1);
             ok = false;
             break;
         }
         const GroupDesc& d = desc[s];
         const int type = d.type, last = d.last;
         if (type != kGrpNone && ((d.need >> x) & 1)) {
-            if (!mbar_wait(&bars.s_full[x], ns & 1, abort)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[x], ns & 1, abort))) {
+                if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxS, g, ns & 1);
                 ok = false;
                 break;
             }
@@ -564,8 +597,13 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
             float mx = v[0];
 #pragma unroll
             for (int c = 1; c < kGroupKeys; ++c) mx = fmaxf(mx, v[c]);
-            if (mx > m + kRescaleThreshold) {
-                const float alpha = ex2(m - mx);  // 0 while m is -inf
+            // Lazy rescale: a row moves its reference max only when the max grew by
+            // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  The
+            // TMEM accesses are .sync.aligned, so the whole warp takes the branch
+            // together; rows that do not need it scale by 1.
+            const bool want = mx > m + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, want)) {
+                const float alpha = want ? ex2(m - mx) : 1.f;  // 0 while m is -inf
                 if (ns > 1) {
                     uint32_t o[32];
 #pragma unroll
@@ -578,7 +616,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                     }
                 }
                 l *= alpha;
-                m = mx;
+                if (want) m = mx;
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
             float rs = 0.f;
@@ -605,7 +643,10 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
 
     // epilogue: O / l -> bf16, lse
     bool have = ns > 0 && ok;
-    if (have) have = mbar_wait(&bars.o_done[x], 0, abort);
+    if (have) {
+        have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[x], 0, abort));
+        if (!have && !*abort) record_wait_failure(p.seq, kSiteSoftmaxO, -1, 0);
+    }
     if (!ok || (ns > 0 && !have)) set_abort(abort, p.err, p.seq);
     tc_fence_after();
     const bool row_ok = i < p.N;
@@ -654,13 +695,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::misc_off + 4);
     uint32_t* patmap = reinterpret_cast<uint32_t*>(sm + L::patmap_off);
 
-    if (*reinterpret_cast<volatile unsigned int*>(&g_abort_seq) == p.seq) return;
     const int n = p.heads.n;
     const int T = p.n_super - 1 - (int)(blockIdx.x / n);  // longest (latest) tiles first
     const int pos = (int)(blockIdx.x % n);
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
+        // one read for the whole CTA: every thread must take the same branch
+        *abort = *reinterpret_cast<volatile unsigned int*>(&g_abort_seq) == p.seq ? 1 : 0;
         mbar_init(bars.q_full, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars.kv_full[s], 1);
@@ -670,9 +712,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars.o_done[s], 1);
         }
         mbar_init(bars.drain, 1);
-        *abort = 0;
         fence_mbar_init();
     }
+    __syncthreads();
+    if (*abort) return;  // an earlier CTA of this launch gave up: skip the work
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -848,6 +891,15 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t read_wait_failure(int* out8) {
+    int rec[8];
+    cudaError_t e = cudaMemcpyFromSymbol(rec, g_wait_fail, sizeof(rec));
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < 8; ++i) out8[i] = rec[i];
+    const int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    return cudaMemcpyToSymbol(g_wait_fail, zero, sizeof(zero));
+}
 
 VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv) {
     VsPrepWs w{};

@@ -107,5 +107,6 @@ struct AttnLaunch {
     int32_t* err_count;
 };
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);
+cudaError_t read_wait_failure(int* out8);
 
 }  // namespace minfer

@@ -87,8 +87,16 @@ typedef struct {
     int window;        /* A-shape: keys i-window+1 .. i kept for row i */
 } mi_params;
 
-/* Stage boundaries recorded by mi_prefill_layer when stage_events != NULL. */
-enum { MI_STAGE_START = 0, MI_STAGE_INDEX_DONE = 1, MI_STAGE_ATTN_DONE = 2, MI_STAGE_EVENTS = 3 };
+/* Stage boundaries recorded by mi_prefill_layer when stage_events != NULL:
+ * START | index kernels | INDEX_DONE | slash/vertical prep | PREP_DONE |
+ * the one sparse-attention launch | ATTN_DONE. */
+enum {
+    MI_STAGE_START = 0,
+    MI_STAGE_INDEX_DONE = 1,
+    MI_STAGE_PREP_DONE = 2,
+    MI_STAGE_ATTN_DONE = 3,
+    MI_STAGE_EVENTS = 4
+};
 
 /* Static description of a status code; never NULL. */
 const char* mi_status_str(int status);
@@ -204,6 +212,17 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
                      int N, int d, float scale, const int8_t* pattern, const mi_params* p,
                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
                      void* stream, void* const* stage_events);
+
+/*
+ * Diagnostics (not on the hot path; synchronous).  The sparse-attention
+ * kernel bounds every wait; the first wait that gives up is recorded as
+ * {launch sequence, site, block, thread, group, parity, 0, 0} with site in
+ * 1..7 (1 producer/stage-free, 2 MMA/Q, 3 MMA/stage-full, 4 MMA/P-ready,
+ * 5 softmax/stage-full, 6 softmax/S-ready, 7 softmax/O-done); site 0 means
+ * no wait gave up.  Reading the record copies it to `record8` (host int32
+ * [8]) and clears it.  A correct run never records anything.
+ */
+int mi_debug_wait_failure(int32_t* record8);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,27 @@
+"""Host-side logic of bench.py: useful-FLOP accounting of a Vertical-Slash
+head, against a brute-force count of the 64x64 tiles and gathered columns."""
+import numpy as np
+
+import bench
+import oracle
+
+
+def brute(v_idx, s_idx, N, d):
+    nB = N // 64
+    D = oracle.slash_deltas(np.asarray(s_idx, np.int32), N).astype(bool)
+    tiles = sum(1 for bq in range(nB) for bk in range(bq + 1) if D[bq - bk])
+    cols = 0
+    for j in sorted(set(int(x) for x in v_idx if 0 <= x < N)):
+        for bq in range(j // 64, nB):
+            if not D[bq - j // 64]:
+                cols += 1
+    return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
+
+
+def test_vs_useful_flops_matches_brute_force():
+    rng = np.random.default_rng(0)
+    for N in (512, 1024, 2048):
+        for _ in range(5):
+            v = rng.integers(-1, N, size=rng.integers(0, 40)).astype(np.int32)
+            s = rng.integers(-1, N, size=rng.integers(0, 30)).astype(np.int32)
+            assert bench.vs_useful_flops(v, s, N, 128) == brute(v, s, N, 128)

@@ -233,5 +233,29 @@ def test_prefill_layer_stage_events_and_stream():
                                     B.make_params(vertical_size=32, slash_size=32),
                                     stage_events=ev, stream=s)
     s.synchronize()
-    assert ev[0].elapsed_time(ev[2]) > 0
+    assert ev[0].elapsed_time(ev[B.MI_STAGE_ATTN_DONE]) > 0
+    assert ev[B.MI_STAGE_PREP_DONE].elapsed_time(ev[B.MI_STAGE_ATTN_DONE]) > 0
     assert torch.isfinite(out.float()).all()
+
+
+def test_single_row_max_jump_rescales_within_warp():
+    """One row's running max jumps by far more than 2^8 mid-stream while its
+    warp neighbours' does not: the lazy O rescale runs for that row only."""
+    N, d = 512, 128
+    q, k, v = rand_bf16(1, 1, N, d, 21)
+    q, k = q.clone(), k.clone()
+    qd = q[0, 300].float()
+    k[0, 256] = (20.0 * qd / qd.norm()).to(torch.bfloat16)  # s(300, 256) ~ 20 * |q|/sqrt(d)
+    every = torch.arange(N, dtype=torch.int32, device="cuda")[None]
+    none = torch.full((1, 1), -1, dtype=torch.int32, device="cuda")
+    out, lse = B.mi_vs_sparse_attn(q, k, v, every, none)
+    torch.cuda.synchronize()
+    qs, ks_, vs_ = head_slices(q, k, v, 0)
+    ro, rl = oracle.attn_dense(qs, ks_, vs_, 0)
+    check_attn(out[0], lse[0], ro, rl)
+
+
+def test_zz_no_device_wait_gave_up():
+    """Every bounded wait of every launch above completed: nothing was recorded."""
+    rec = B.mi_debug_wait_failure()
+    assert rec["site"] == 0, rec
