@@ -30,7 +30,8 @@ MI_BLOCK = 64
 # every symbol include/minfer.h declares
 EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
-           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure"]
+           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
+           "mi_vs_index_static"]
 
 
 class MinferError(RuntimeError):
@@ -77,6 +78,7 @@ def _lib_handle():
         lib.mi_prefill_layer.argtypes = [P, P, P, I, I, I, I, F, P, ctypes.POINTER(mi_params),
                                          P, P, P, P, SZ, P, P]
         lib.mi_debug_wait_failure.argtypes = [P]
+        lib.mi_vs_index_static.argtypes = [P, P, I, I, I, I, F, I, I, I, P, I, P, P, P, P, P]
         for name in EXPORTS[5:]:
             getattr(lib, name).restype = I
         _lib = lib
@@ -172,6 +174,24 @@ def mi_vs_index(q, k, last_q, vertical_size, slash_size, heads: Optional[Sequenc
                                    slash_size, hp, n, _ptr(v_idx), _ptr(s_idx), _ptr(vs), _ptr(ss),
                                    _ptr(ws), ws.numel(), _stream(stream))
     _check("mi_vs_index", rc)
+    return (v_idx, s_idx, vs, ss) if want_scores else (v_idx, s_idx)
+
+
+def mi_vs_index_static(q, k, last_q, vertical_size, slash_size, heads=None, scale=0.0,
+                       want_scores=False, stream=None):
+    """mi_vs_index for callers that cannot provide a workspace: the library keeps
+    the scratch in a fixed 16 MiB device array (calls must not overlap)."""
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    dev = q.device
+    v_idx = torch.empty(n, vertical_size, dtype=torch.int32, device=dev)
+    s_idx = torch.empty(n, slash_size, dtype=torch.int32, device=dev)
+    vs = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    ss = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    rc = _lib_handle().mi_vs_index_static(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, last_q,
+                                          vertical_size, slash_size, hp, n, _ptr(v_idx),
+                                          _ptr(s_idx), _ptr(vs), _ptr(ss), _stream(stream))
+    _check("mi_vs_index_static", rc)
     return (v_idx, s_idx, vs, ss) if want_scores else (v_idx, s_idx)
 
 

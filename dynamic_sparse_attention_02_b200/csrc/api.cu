@@ -11,14 +11,17 @@
 using namespace minfer;
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
+}  // namespace
 
-int cuda_status(cudaError_t e) {
+// MI_OK, or MI_ERR_CUDA with the error kept for mi_last_cuda_error().
+int minfer::cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return MI_OK;
     g_last_cuda_error = (int)e;
     return MI_ERR_CUDA;
 }
+
+namespace {
 
 // Shapes every entry point shares.  Fills `hl` with the listed heads
 // (pattern and per-pattern position filled by the caller).

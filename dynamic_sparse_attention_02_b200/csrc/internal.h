@@ -109,4 +109,7 @@ struct AttnLaunch {
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);
 cudaError_t read_wait_failure(int* out8);
 
+// MI_OK, or MI_ERR_CUDA with the error kept for mi_last_cuda_error().
+int cuda_status(cudaError_t e);
+
 }  // namespace minfer

@@ -214,6 +214,32 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
                      void* stream, void* const* stage_events);
 
 /*
+ * mi_vs_index without a workspace argument.  The paper has no counterpart:
+ * this entry point exists for callers that cannot provide device scratch --
+ * e.g. an inference server that reserves nearly all HBM for its KV-cache pool
+ * and forbids new allocations on the request path, or host code on a
+ * latency-critical path where cudaMalloc's implicit synchronisation is not
+ * acceptable.  It computes exactly what mi_vs_index computes (same kernels,
+ * same results), with its scratch in a 16 MiB array inside the library that
+ * every GPU which loads the library holds until the process exits.  It
+ * allocates nothing.
+ *  - Capacity: the call needs the bytes mi_workspace_bytes(MI_OP_VS_INDEX,
+ *    ...) reports for the same arguments; beyond 16 MiB it returns
+ *    MI_ERR_UNSUPPORTED and launches nothing (for example 8 heads at
+ *    N = 131072 fit, 32 heads at N = 131072 do not).
+ *  - Every call shares that one array.  Calls whose work overlaps on the GPU
+ *    (other streams, other host threads, concurrent graph replays) race on
+ *    it; serialise them, e.g. on one stream.
+ *  - The first call on each device looks up the array's device address and
+ *    caches it; make that first call before any stream capture on the device.
+ * All other arguments, outputs and errors as for mi_vs_index.
+ */
+int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d,
+                       float scale, int last_q, int vertical_size, int slash_size,
+                       const int32_t* heads, int n_heads, int32_t* v_idx, int32_t* s_idx,
+                       float* v_score, float* s_score, void* stream);
+
+/*
  * Diagnostics (not on the hot path; synchronous).  The sparse-attention
  * kernel bounds every wait; the first wait that gives up is recorded as
  * {launch sequence, site, block, thread, group, parity, 0, 0} with site in

@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = header_functions()
-    assert len(names) == 12
+    assert len(names) == 13
     assert sorted(B.EXPORTS) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -130,3 +130,16 @@ def test_workspace_queries(lib):
     vs_only = B.mi_prefill_workspace_bytes(32, 8, 131072, 128, np.ones(32, np.int8), p)
     a_only = B.mi_prefill_workspace_bytes(32, 8, 131072, 128, np.zeros(32, np.int8), p)
     assert full >= vs_only > a_only >= 0
+
+
+def test_vs_index_static_validation_and_capacity(lib):
+    """The no-workspace entry point validates like mi_vs_index and rejects
+    shapes whose scratch exceeds its fixed array -- both before any CUDA call."""
+    f = FAKE
+    assert lib.mi_vs_index_static(None, f, 4, 2, 512, 128, 0.0, 64, 16, 32, None, 0, f, f, None,
+                                  None, None) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_vs_index_static(f, f, 4, 2, 500, 128, 0.0, 64, 16, 32, None, 0, f, f, None,
+                                  None, None) == B.MI_ERR_UNSUPPORTED
+    # 32 heads at N = 131072 need 36 MiB of scratch: more than the 16 MiB array
+    assert lib.mi_vs_index_static(f, f, 32, 8, 131072, 128, 0.0, 64, 1000, 6096, None, 0, f, f,
+                                  None, None, None) == B.MI_ERR_UNSUPPORTED
