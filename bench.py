@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="minfer", choices=["minfer", "reference"])
     ap.add_argument("--workload", default="vs_n128k_llama3_8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override N of the workload (smaller profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
@@ -220,11 +222,16 @@ def rows_for_budget(w, budget_s):
 
 # ----------------------------------------------------------------- arms
 
+def workload_of(args):
+    w = synth.workload(args.workload)
+    return synth.workload(args.workload, N=args.seq_len) if args.seq_len else w
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = synth.workload(args.workload)
+    w = workload_of(args)
     x = synth.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     rng = np.random.default_rng(w.seed)
     total = args.steps + args.warmup
@@ -253,7 +260,8 @@ def config_of(w):
             "pattern": w.pattern, "last_q": w.last_q, "vertical_size": w.vertical_size,
             "slash_size": w.slash_size, "topk_blocks": w.topk_blocks, "sink": w.sink,
             "window": w.window, "parallelism": "replicas",
-            "l2": "inputs larger than L2 (q 1 GiB, k+v 512 MiB at 128K); no flush"}
+            "l2": (f"inputs larger than L2 (q+k+v {(w.Hq + 2 * w.Hkv) * w.N * w.d * 2 / 2**20:.0f} MiB"
+                   " > 126 MB); no flush")}
 
 
 def run_minfer(args):
@@ -282,8 +290,8 @@ def run_minfer(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = synth.workload(args.workload)
-    log(f"generating {w.name}")
+    w = workload_of(args)
+    log(f"generating {w.name} (N={w.N})")
     x = synth.make_inputs(w, device=str(dev))
     torch.cuda.synchronize()
     q, k, v = x["q"], x["k"], x["v"]

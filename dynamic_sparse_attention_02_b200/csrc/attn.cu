@@ -36,9 +36,17 @@ namespace minfer {
 
 namespace {
 
-constexpr int kThreads = 320;
+// 3 warpgroups: two softmax warpgroups (one per 128-row slot) and one for the
+// producer warp, the MMA warp and two idle warps.  Launched at 168 registers
+// per thread (65536 / 384, rounded down to 8); the softmax warpgroups then
+// take 224 and the third gives back down to 56: 2*128*224 + 128*56 = 384*168.
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168,
+              "register split exceeds the launch budget");
 constexpr int kSoftmaxThreads = 256;
 constexpr int kGroupKeys = 128;
 constexpr int kPanelBytes = 128 * 128;  // 128 rows x one 64-column (128-byte) panel
@@ -566,7 +574,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                 for (int c = 0; c < 4; ++c) {
                     tmem_ld32(tS + 32 * c, r);
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) v[32 * c + u] = __uint_as_float(r[u]) * p.scale_log2;
+                    for (int u = 0; u < 32; ++u) v[32 * c + u] = __uint_as_float(r[u]);
                 }
             }
             if (type == kGrpTiles) {
@@ -594,9 +602,13 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                     if (!keep) v[c] = -INFINITY;
                 }
             }
+            // raw scores: the scale (> 0) commutes with the max and is folded into
+            // the exponent below, one FFMA per element
+            const float cs = p.scale_log2;
             float mx = v[0];
 #pragma unroll
             for (int c = 1; c < kGroupKeys; ++c) mx = fmaxf(mx, v[c]);
+            mx *= cs;
             // Lazy rescale: a row moves its reference max only when the max grew by
             // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  The
             // TMEM accesses are .sync.aligned, so the whole warp takes the branch
@@ -625,8 +637,8 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                 uint32_t pk[32];
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                    const float p0 = ex2(v[64 * c + 2 * u] - mu);
-                    const float p1 = ex2(v[64 * c + 2 * u + 1] - mu);
+                    const float p0 = ex2(fmaf(v[64 * c + 2 * u], cs, -mu));
+                    const float p1 = ex2(fmaf(v[64 * c + 2 * u + 1], cs, -mu));
                     rs += p0 + p1;
                     pk[u] = pack_bf16(p0, p1);
                 }
@@ -726,13 +738,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp < 8) {
+        regs_inc<kSoftmaxRegs>();
         run_softmax<D>(p, sm, bars, abort, tmem, pos, T);
-    } else if (warp == kProducerWarp) {
-        run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
     } else {
-        if ((threadIdx.x & 31) == 0) run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
-        __syncwarp();
-        tc_fence_before();
+        regs_dec<kControlRegs>();
+        if (warp == kProducerWarp) {
+            run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
+        } else if (warp == kMmaWarp) {
+            if ((threadIdx.x & 31) == 0) run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
+            __syncwarp();
+            tc_fence_before();
+        }
     }
     __syncthreads();
     if (warp == kMmaWarp) {
