@@ -62,7 +62,7 @@ def parse_args():
                     help="override N of the workload (smaller profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget-s", type=float, default=20.0,
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0,
                     help="approximate CPU seconds for the oracle baseline sample")
     return ap.parse_args()
 
@@ -175,25 +175,27 @@ def vs_useful_flops(v_idx, s_idx, N, d):
 
 # ----------------------------------------------------------------- oracle timing
 
-def oracle_sample(w, x, n_rows, rng, heads=(0,)):
-    """Time the CPU oracle on a bounded sample; returns (extrapolated ms/layer, desc, cores)."""
+def oracle_sample(w, x, budget_s, rng, h=0, min_rows=32, max_rows=16384):
+    """Time the CPU oracle on a bounded sample of head h: its index, then seeded
+    random rows of its attention in chunks until `budget_s` of CPU time is used.
+    Returns (extrapolated ms/layer, description, threads used)."""
     import oracle
     pattern = x["pattern"]
-    t_index = 0.0
-    t_rows = 0.0
-    rows_done = 0
-    for h in heads:
-        g = h * w.Hkv // w.Hq
-        qs = x["q"][h:h + 1].float().cpu()
-        ks = x["k"][g:g + 1].float().cpu()
-        vs = x["v"][g:g + 1].float().cpu()
-        rows = np.sort(rng.choice(w.N, size=n_rows, replace=False))
-        pt = int(pattern[h])
-        t0 = time.perf_counter()
-        if pt == synth.PATTERN_VS:
-            vi, si, _, _ = oracle.vs_index(qs, ks, 0, w.last_q, w.vertical_size, w.slash_size)
-        elif pt == synth.PATTERN_BS:
-            bi, bc = oracle.bs_index(qs, ks, 0, w.topk_blocks)
+    g = h * w.Hkv // w.Hq
+    qs = x["q"][h:h + 1].float().cpu()
+    ks = x["k"][g:g + 1].float().cpu()
+    vs = x["v"][g:g + 1].float().cpu()
+    pt = int(pattern[h])
+    t0 = time.perf_counter()
+    if pt == synth.PATTERN_VS:
+        vi, si, _, _ = oracle.vs_index(qs, ks, 0, w.last_q, w.vertical_size, w.slash_size)
+    elif pt == synth.PATTERN_BS:
+        bi, bc = oracle.bs_index(qs, ks, 0, w.topk_blocks)
+    t_index = time.perf_counter() - t0
+    order = rng.permutation(w.N)
+    t_rows, done, chunk = 0.0, 0, min_rows
+    while done < min(max_rows, w.N) and (done < min_rows or t_index + t_rows < budget_s):
+        rows = np.sort(order[done:done + chunk])
         t1 = time.perf_counter()
         if pt == synth.PATTERN_VS:
             oracle.attn_vs(qs, ks, vs, 0, vi, si, rows=rows)
@@ -201,23 +203,13 @@ def oracle_sample(w, x, n_rows, rng, heads=(0,)):
             oracle.attn_bs(qs, ks, vs, 0, bi, bc, rows=rows)
         else:
             oracle.attn_ashape(qs, ks, vs, 0, w.sink, w.window, rows=rows)
-        t2 = time.perf_counter()
-        t_index += t1 - t0
-        t_rows += t2 - t1
-        rows_done += n_rows
-    nh = len(heads)
-    ms = 1e3 * (t_index / nh * w.Hq + t_rows / rows_done * w.N * w.Hq)
-    desc = (f"index of {nh} head(s) + {n_rows} seeded random rows of attention per head at "
-            f"N={w.N}, extrapolated to {w.Hq} heads x {w.N} rows")
+        t_rows += time.perf_counter() - t1
+        done += rows.size
+        chunk = min(2 * chunk, 2048)
+    ms = 1e3 * (t_index * w.Hq + t_rows / done * w.N * w.Hq)
+    desc = (f"index of head {h} ({t_index:.1f} s) + {done} seeded random rows of its attention "
+            f"at N={w.N} ({t_rows:.1f} s), extrapolated to {w.Hq} heads x {w.N} rows")
     return ms, desc, oracle.num_threads()
-
-
-def rows_for_budget(w, budget_s):
-    # ~4*d*N/2 flops per row in fp64 loops at ~1 GFLOP/s per core, plus the index
-    import oracle
-    cores = max(1, oracle.num_threads())
-    per_row = 4.0 * w.d * w.N / 2 / (1.0e9 * cores)
-    return int(min(2048, max(16, budget_s * 0.6 / max(per_row, 1e-9))))
 
 
 # ----------------------------------------------------------------- arms
@@ -235,13 +227,13 @@ def run_reference(args):
     x = synth.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     rng = np.random.default_rng(w.seed)
     total = args.steps + args.warmup
-    n_rows = max(16, rows_for_budget(w, 150.0 / max(total, 1)) // 2)
+    budget = max(2.0, 150.0 / max(total, 1))  # the whole run stays within a few minutes
     for _ in range(args.warmup):
-        oracle_sample(w, x, n_rows, rng)
+        oracle_sample(w, x, budget, rng)
     vals = []
     desc, cores = "", 1
     for _ in range(args.steps):
-        ms, desc, cores = oracle_sample(w, x, n_rows, rng)
+        ms, desc, cores = oracle_sample(w, x, budget, rng)
         vals.append(ms)
     v = float(np.median(vals))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
@@ -396,10 +388,9 @@ def run_minfer(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             rng = np.random.default_rng(w.seed)
-            n_rows = rows_for_budget(w, args.cpu_budget_s)
-            log(f"oracle baseline: {n_rows} rows")
-            ms_cpu, desc, cores = oracle_sample(w, x, n_rows, rng)
-            log("oracle baseline done")
+            log(f"oracle baseline: ~{args.cpu_budget_s:.0f} s of CPU work")
+            ms_cpu, desc, cores = oracle_sample(w, x, args.cpu_budget_s, rng)
+            log("oracle baseline done: " + desc)
             cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                    "sample": desc}
         line = {
