@@ -29,6 +29,7 @@
 #include <cstring>
 #include <cudaTypedefs.h>
 
+#include "exp2_poly.h"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -114,7 +115,9 @@ struct AttnParams {
     int topk;
     int sink, window;
     int32_t* err;
-    HeadList heads;
+    HeadList heads;  // sorted by KV head
+    int ngroups;     // KV heads present in `heads`
+    uint16_t grp_start[MI_MAX_HEADS + 1];  // heads of KV group i: [grp_start[i], grp_start[i+1])
 };
 
 template <int D>
@@ -124,10 +127,11 @@ struct Layout {
     static constexpr int q_off = 0;
     static constexpr int k_off = q_off + 2 * kQBytes;
     static constexpr int v_off = k_off + 2 * kKVBytes;
+    static constexpr int kDescRing = 4;  // group descriptors in flight
     static constexpr int desc_off = v_off + 2 * kKVBytes;
-    static constexpr int held_off = desc_off + 2 * (int)sizeof(GroupDesc);
+    static constexpr int held_off = desc_off + kDescRing * (int)sizeof(GroupDesc);
     static constexpr int bar_off = (held_off + (int)sizeof(GatherHeld) + 15) & ~15;
-    static constexpr int kNumBars = 12;
+    static constexpr int kNumBars = 24;
     static constexpr int misc_off = bar_off + kNumBars * 8;
     static constexpr int patmap_off = misc_off + 16;
     static size_t bytes(int patmap_words) {
@@ -138,13 +142,21 @@ struct Layout {
     }
 };
 
+// Pipeline barriers.  Group g (in publication order) uses descriptor slot
+// g % 4 and, if it carries keys, K stage and V stage g % 2.  K is released as
+// soon as the S = Q K^T of its group has run, V only after P V, so the next
+// K tile streams in while the current P V is still pending.
 struct Bars {
     uint64_t* q_full;
-    uint64_t* kv_full;   // [2]
-    uint64_t* kv_empty;  // [2]
-    uint64_t* s_full;    // [2]
-    uint64_t* p_full;    // [2]
-    uint64_t* o_done;    // [2]
+    uint64_t* desc_full;   // [4] producer -> MMA, softmax
+    uint64_t* desc_empty;  // [4] MMA + 256 softmax threads -> producer
+    uint64_t* k_full;      // [2] TMA / gather -> MMA
+    uint64_t* k_empty;     // [2] MMA (after S) -> producer
+    uint64_t* v_full;      // [2]
+    uint64_t* v_empty;     // [2] MMA (after P V) -> producer
+    uint64_t* s_full;      // [2] per slot: S ready in TMEM
+    uint64_t* p_full;      // [2] per slot: P written to TMEM
+    uint64_t* o_done;      // [2] per slot: last P V done
     uint64_t* drain;
 };
 
@@ -152,6 +164,51 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---- packed fp32 pairs (one 64-bit register pair, two lanes of work)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair on the FMA pipe (method and error bound in exp2_poly.h).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, kExp2Clamp), fmaxf(x1, kExp2Clamp));
+    const uint64_t t = f2_add(xc, f2_pack(kExp2Round, kExp2Round));        // round to nearest
+    const uint64_t n = f2_add(t, f2_pack(-kExp2Round, -kExp2Round));       // n as float
+    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);                 // x - n, exact
+    uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+    q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    // n sits in the low mantissa bits of t; (bits(t) << 23) adds n to the exponent
+    const float r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    const float r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+    return f2_pack(r0, r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -177,94 +234,126 @@ struct Producer {
     volatile int* abort;
     GroupDesc* desc;
     GatherHeld* held;
-    int g;       // KV head
-    int pub = 0; // groups published
+    int g;        // KV head
+    int pub = 0;  // descriptors published
+    int nk = 0;   // K stages filled
+    int nv = 0;   // V stages filled
     int lane;
     bool ok = true;
 
-    __device__ bool acquire(int& s) {
-        s = pub & 1;
-        if (pub >= 2) {
-            bool w = true;
-            if (lane == 0) w = mbar_wait(&bars.kv_empty[s], ((pub >> 1) - 1) & 1, abort);
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (!w) {
-                if (lane == 0) {
-                    if (!*abort) record_wait_failure(p.seq, kSiteProducerEmpty, pub, ((pub >> 1) - 1) & 1);
-                    set_abort(abort, p.err, p.seq);
-                }
-                ok = false;
-                return false;
+    // lane 0 waits, the warp follows its verdict
+    __device__ bool wait(uint64_t* bar, int parity, int count) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(bar, parity, abort);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+            if (lane == 0) {
+                if (!*abort) record_wait_failure(p.seq, kSiteProducerEmpty, count, parity);
+                set_abort(abort, p.err, p.seq);
             }
+            ok = false;
         }
-        return true;
+        return w;
+    }
+    __device__ GroupDesc* acquire_desc() {
+        const int i = pub & (L::kDescRing - 1);
+        if (pub >= L::kDescRing && !wait(&bars.desc_empty[i], ((pub / L::kDescRing) - 1) & 1, pub))
+            return nullptr;
+        return &desc[i];
+    }
+    __device__ void publish_desc() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.desc_full[pub & (L::kDescRing - 1)]);
+        ++pub;
+    }
+    __device__ bool acquire_k(int& s) {
+        s = nk & 1;
+        return nk < 2 || wait(&bars.k_empty[s], ((nk >> 1) - 1) & 1, nk);
+    }
+    __device__ bool acquire_v(int& s) {
+        s = nv & 1;
+        return nv < 2 || wait(&bars.v_empty[s], ((nv >> 1) - 1) & 1, nv);
     }
 
     __device__ void tiles(int b0, int m0, int b1, int m1) {
         if (!ok) return;
-        int s;
-        if (!acquire(s)) return;
+        GroupDesc* d = acquire_desc();
+        if (!d) return;
         if (lane == 0) {
-            GroupDesc& d = desc[s];
-            d.type = kGrpTiles;
-            d.last = 0;
-            d.need = (((m0 | m1) & 0x3) ? 1 : 0) | (((m0 | m1) & 0xC) ? 2 : 0);
-            d.ncols = 0;
-            d.b0 = b0;
-            d.b1 = b1;
-            d.m0 = m0;
-            d.m1 = m1;
-            mbar_arrive_expect_tx(&bars.kv_full[s], 2 * L::kKVBytes);
-            uint8_t* kd = sm + L::k_off + s * L::kKVBytes;
-            uint8_t* vd = sm + L::v_off + s * L::kKVBytes;
+            d->type = kGrpTiles;
+            d->last = 0;
+            d->need = (((m0 | m1) & 0x3) ? 1 : 0) | (((m0 | m1) & 0xC) ? 2 : 0);
+            d->ncols = 0;
+            d->b0 = b0;
+            d->b1 = b1;
+            d->m0 = m0;
+            d->m1 = m1;
+        }
+        publish_desc();
+        const int row0 = g * p.N + 64 * b0, row1 = g * p.N + 64 * b1;
+        int sk;
+        if (!acquire_k(sk)) return;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bars.k_full[sk], L::kKVBytes);
+            uint8_t* kd = sm + L::k_off + sk * L::kKVBytes;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = g * p.N + 64 * (h ? b1 : b0);
-#pragma unroll
-                for (int pn = 0; pn < D / 64; ++pn) {
-                    tma_load_2d(kd + pn * kPanelBytes + h * (kPanelBytes / 2), tmK, 64 * pn, row,
-                                &bars.kv_full[s]);
-                    tma_load_2d(vd + pn * kPanelBytes + h * (kPanelBytes / 2), tmV, 64 * pn, row,
-                                &bars.kv_full[s]);
-                }
+            for (int pn = 0; pn < D / 64; ++pn) {
+                tma_load_2d(kd + pn * kPanelBytes, tmK, 64 * pn, row0, &bars.k_full[sk]);
+                tma_load_2d(kd + pn * kPanelBytes + kPanelBytes / 2, tmK, 64 * pn, row1,
+                            &bars.k_full[sk]);
             }
         }
         __syncwarp();
-        ++pub;
+        ++nk;
+        int sv;
+        if (!acquire_v(sv)) return;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bars.v_full[sv], L::kKVBytes);
+            uint8_t* vd = sm + L::v_off + sv * L::kKVBytes;
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn) {
+                tma_load_2d(vd + pn * kPanelBytes, tmV, 64 * pn, row0, &bars.v_full[sv]);
+                tma_load_2d(vd + pn * kPanelBytes + kPanelBytes / 2, tmV, 64 * pn, row1,
+                            &bars.v_full[sv]);
+            }
+        }
+        __syncwarp();
+        ++nv;
     }
 
     __device__ void gather(int n) {
         if (!ok) return;
-        int s;
-        if (!acquire(s)) return;
-        GroupDesc& d = desc[s];
+        GroupDesc* d = acquire_desc();
+        if (!d) return;
         int need = 0;
         for (int c = lane; c < kGroupKeys; c += 32) {
             const bool v = c < n;
             const int col = v ? held->cols[c] : held->cols[0];
             const int cm = v ? held->cm[c] : 0;
-            d.cols[c] = col;
-            d.cm[c] = (uint8_t)cm;
+            d->cols[c] = col;
+            d->cm[c] = (uint8_t)cm;
             need |= cm;
         }
         for (int off = 16; off >= 1; off >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, off);
         if (lane == 0) {
-            d.type = kGrpGather;
-            d.last = 0;
-            d.need = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
-            d.ncols = n;
-            d.b0 = d.b1 = -1;
-            d.m0 = d.m1 = 0;
+            d->type = kGrpGather;
+            d->last = 0;
+            d->need = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
+            d->ncols = n;
+            d->b0 = d->b1 = -1;
+            d->m0 = d->m1 = 0;
         }
-        __syncwarp();
-        uint8_t* kd = sm + L::k_off + s * L::kKVBytes;
-        uint8_t* vd = sm + L::v_off + s * L::kKVBytes;
+        publish_desc();
+        int sk, sv;
+        if (!acquire_k(sk) || !acquire_v(sv)) return;
+        uint8_t* kd = sm + L::k_off + sk * L::kKVBytes;
+        uint8_t* vd = sm + L::v_off + sv * L::kKVBytes;
         constexpr int kChunks = D / 8;  // 16-byte chunks per row
         const bf16* kb = p.k + (size_t)g * p.N * D;
         const bf16* vb = p.v + (size_t)g * p.N * D;
         for (int idx = lane; idx < kGroupKeys * kChunks; idx += 32) {
             const int r = idx / kChunks, c = idx % kChunks;
-            const size_t src = (size_t)d.cols[r] * D + c * 8;
+            const size_t src = (size_t)d->cols[r] * D + c * 8;
             const int dst = (c >> 3) * kPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
             cp_async_16(kd + dst, kb + src);
             cp_async_16(vd + dst, vb + src);
@@ -272,34 +361,35 @@ struct Producer {
         cp_async_wait_all();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.kv_full[s]);
-        ++pub;
+        if (lane == 0) {
+            mbar_arrive(&bars.k_full[sk]);
+            mbar_arrive(&bars.v_full[sv]);
+        }
+        ++nk;
+        ++nv;
     }
 
     __device__ void finish() {
         if (!ok) return;
-        int s;
-        if (!acquire(s)) return;
+        GroupDesc* d = acquire_desc();
+        if (!d) return;
         if (lane == 0) {
-            GroupDesc& d = desc[s];
-            d.type = kGrpNone;
-            d.last = 1;
-            d.need = 0;
-            d.ncols = 0;
-            mbar_arrive(&bars.kv_full[s]);
+            d->type = kGrpNone;
+            d->last = 1;
+            d->need = 0;
+            d->ncols = 0;
         }
-        __syncwarp();
-        ++pub;
+        publish_desc();
     }
 
     // Wait (bounded) until every copy this warp started has landed, so that
     // no TMA write can reach shared memory after the CTA exits.
     __device__ void drain() {
         if (lane != 0) return;
-        for (int u = pub - 2; u < pub; ++u) {
-            if (u < 0) continue;
-            mbar_wait_budget(&bars.kv_full[u & 1], (u >> 1) & 1);
-        }
+        for (int u = nk - 2; u < nk; ++u)
+            if (u >= 0) mbar_wait_budget(&bars.k_full[u & 1], (u >> 1) & 1);
+        for (int u = nv - 2; u < nv; ++u)
+            if (u >= 0) mbar_wait_budget(&bars.v_full[u & 1], (u >> 1) & 1);
     }
 };
 
@@ -450,58 +540,78 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
 }
 
 // ------------------------------------------------------------- MMA issuer
+// The whole warp runs this loop converged: bookkeeping and descriptors are
+// uniform, lane 0 alone polls the barriers and broadcasts the outcome, and
+// elect.sync inside the issue instructions picks the single issuing lane.
 template <int D>
 __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int32_t* err,
                         unsigned int seq, uint32_t tmem) {
     using L = Layout<D>;
+    const int lane = threadIdx.x & 31;
     const uint32_t idS = idesc_bf16_f32(128, kGroupKeys, false);
     const uint32_t idO = idesc_bf16_f32(128, D, true);
     const uint32_t q_addr = smem_u32(sm + L::q_off);
     const uint32_t k_addr = smem_u32(sm + L::k_off);
     const uint32_t v_addr = smem_u32(sm + L::v_off);
     const GroupDesc* desc = reinterpret_cast<const GroupDesc*>(sm + L::desc_off);
+    auto wait = [&](uint64_t* bar, int parity) -> bool {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(bar, parity, abort);
+        return __shfl_sync(0xffffffffu, w, 0);
+    };
 
-    int pend[2] = {-1, -1}, pend_stage[2] = {0, 0}, npv[2] = {0, 0}, np[2] = {0, 0};
-    int uses[2] = {0, 0};
-    bool ok = mbar_wait(bars.q_full, 0, abort);
-    if (!ok && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, 0);
+    int pend[2] = {-1, -1}, npv[2] = {0, 0}, np[2] = {0, 0};
+    int vuses[2] = {0, 0};
+    bool ok = wait(bars.q_full, 0);
+    if (!ok && lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, 0);
     int g = 0;
     while (ok) {
-        const int s = g & 1;
-        if (!mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort)) {
-            if (!*abort) record_wait_failure(seq, kSiteMmaFull, g, (g >> 1) & 1);
+        const int di = g & (L::kDescRing - 1);
+        if (!wait(&bars.desc_full[di], (g / L::kDescRing) & 1)) {
+            if (lane == 0 && !*abort)
+                record_wait_failure(seq, kSiteMmaFull, g, (g / L::kDescRing) & 1);
             ok = false;
             break;
         }
-        tc_fence_after();
-        const int type = desc[s].type, need = desc[s].need, last = desc[s].last;
-        if (type == kGrpNone)
-            mbar_arrive(&bars.kv_empty[s]);
-        else
-            uses[s] = __popc(need);
+        const int type = desc[di].type, need = desc[di].need, last = desc[di].last;
+        const int s = g & 1;  // data groups are numbered like descriptors (the end marker is last)
+        bool k_ready = false;
+        // per slot: first the pending O += P V (needs only P and V), then S of
+        // this group (needs K): a late K tile does not hold back the other work
         for (int x = 0; x < 2 && ok; ++x) {
             if (pend[x] >= 0) {
-                if (!mbar_wait(&bars.p_full[x], np[x] & 1, abort)) {
-                    if (!*abort) record_wait_failure(seq, kSiteMmaP, g, np[x] & 1);
+                // P of the slot's previous group, then its V: issue O += P V
+                const int pg = pend[x], st = pg & 1;
+                if (!wait(&bars.p_full[x], np[x] & 1) || !wait(&bars.v_full[st], (pg >> 1) & 1)) {
+                    if (lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaP, g, np[x] & 1);
                     ok = false;
                     break;
                 }
                 ++np[x];
                 tc_fence_after();
-                const int st = pend_stage[x];
                 const uint32_t tP = tmem + 256 * x;
                 const uint32_t tO = tmem + 256 * x + 128;
 #pragma unroll
                 for (int kk = 0; kk < kGroupKeys / 16; ++kk) {
                     const uint64_t bdesc =
                         sw128_desc(v_addr + st * L::kKVBytes + kk * 2048, kPanelBytes, 1024);
-                    mma_ts(tO, tP + kk * 8, bdesc, idO, (npv[x] > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts_warp(tO, tP + kk * 8, bdesc, idO, (npv[x] > 0 || kk > 0) ? 1u : 0u);
                 }
                 ++npv[x];
-                if (--uses[st] == 0) mma_commit(&bars.kv_empty[st]);
+                if (--vuses[st] == 0) mma_commit_warp(&bars.v_empty[st]);
                 pend[x] = -1;
             }
             if (type != kGrpNone && ((need >> x) & 1)) {
+                if (!k_ready) {
+                    if (!wait(&bars.k_full[s], (g >> 1) & 1)) {
+                        if (lane == 0 && !*abort)
+                            record_wait_failure(seq, kSiteMmaFull, g, (g >> 1) & 1);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    k_ready = true;
+                }
                 const uint32_t tS = tmem + 256 * x;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -510,22 +620,28 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
                         sw128_desc(q_addr + x * L::kQBytes + pn * kPanelBytes + off, 16, 1024);
                     const uint64_t bdesc =
                         sw128_desc(k_addr + s * L::kKVBytes + pn * kPanelBytes + off, 16, 1024);
-                    mma_ss(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
+                    mma_ss_warp(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars.s_full[x]);
+                mma_commit_warp(&bars.s_full[x]);
                 pend[x] = g;
-                pend_stage[x] = s;
             }
         }
-        if (!ok || last) break;
+        if (!ok) break;
+        if (type != kGrpNone) {
+            mma_commit_warp(&bars.k_empty[s]);  // K free once this group's S has run
+            vuses[s] = __popc(need);
+        }
+        mbar_arrive_warp(&bars.desc_empty[di]);
+        if (last) break;
         ++g;
     }
-    if (!ok) set_abort(abort, err, seq);
+    if (!ok && lane == 0) set_abort(abort, err, seq);
     for (int x = 0; x < 2; ++x)
-        if (npv[x] > 0) mma_commit(&bars.o_done[x]);
+        if (npv[x] > 0) mma_commit_warp(&bars.o_done[x]);
     // every MMA must have finished before TMEM is released
-    mma_commit(bars.drain);
-    mbar_wait_budget(bars.drain, 0);
+    mma_commit_warp(bars.drain);
+    if (lane == 0) mbar_wait_budget(bars.drain, 0);
+    __syncwarp();
 }
 
 // ------------------------------------------------------------- softmax
@@ -551,13 +667,14 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     int ns = 0;
     bool ok = true;
     for (int g = 0;; ++g) {
-        const int s = g & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.kv_full[s], (g >> 1) & 1, abort))) {
-            if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxFull, g, (g >> 1) & 1);
+        const int di = g & (L::kDescRing - 1);
+        const int dpar = (g / L::kDescRing) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.desc_full[di], dpar, abort))) {
+            if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxFull, g, dpar);
             ok = false;
             break;
         }
-        const GroupDesc& d = desc[s];
+        const GroupDesc& d = desc[di];
         const int type = d.type, last = d.last;
         if (type != kGrpNone && ((d.need >> x) & 1)) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[x], ns & 1, abort))) {
@@ -569,13 +686,10 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
             tc_fence_after();
             float v[kGroupKeys];
             {
-                uint32_t r[32];
+                uint32_t r[kGroupKeys];
+                tmem_ld128(tS, r);  // the whole row of S: one TMEM round trip
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tS + 32 * c, r);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) v[32 * c + u] = __uint_as_float(r[u]);
-                }
+                for (int u = 0; u < kGroupKeys; ++u) v[u] = __uint_as_float(r[u]);
             }
             if (type == kGrpTiles) {
 #pragma unroll
@@ -603,11 +717,18 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                 }
             }
             // raw scores: the scale (> 0) commutes with the max and is folded into
-            // the exponent below, one FFMA per element
+            // the exponent below (one packed FFMA per pair)
             const float cs = p.scale_log2;
-            float mx = v[0];
+            // four independent max chains (latency), then combined
+            float mq[4] = {fmaxf(v[0], v[1]), fmaxf(v[2], v[3]), fmaxf(v[4], v[5]),
+                           fmaxf(v[6], v[7])};
 #pragma unroll
-            for (int c = 1; c < kGroupKeys; ++c) mx = fmaxf(mx, v[c]);
+            for (int c = 8; c < kGroupKeys; c += 8) {
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4)
+                    mq[w4] = fmax3(mq[w4], v[c + 2 * w4], v[c + 2 * w4 + 1]);
+            }
+            float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
             mx *= cs;
             // Lazy rescale: a row moves its reference max only when the max grew by
             // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  The
@@ -631,25 +752,38 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                 if (want) m = mx;
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
-            float rs = 0.f;
+            const uint64_t cs2 = f2_pack(cs, cs), nmu2 = f2_pack(-mu, -mu);
+            // four independent packed row-sum accumulators (latency)
+            uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f),
+                                f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                    const float p0 = ex2(fmaf(v[64 * c + 2 * u], cs, -mu));
-                    const float p1 = ex2(fmaf(v[64 * c + 2 * u + 1], cs, -mu));
-                    rs += p0 + p1;
+                    const uint64_t x2 =
+                        f2_fma(f2_pack(v[64 * c + 2 * u], v[64 * c + 2 * u + 1]), cs2, nmu2);
+                    // all exponentials on MUFU: measured faster than moving a share to
+                    // the FMA pipe, the softmax warp is bound by its own issue rate
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+                    sum2[u & 3] = f2_add(sum2[u & 3], p2);
+                    float p0, p1;
+                    f2_unpack(p2, p0, p1);
                     pk[u] = pack_bf16(p0, p1);
                 }
                 tmem_st32(tS + 32 * c, pk);
             }
+            float s0, s1;
+            f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+            const float rs = s0 + s1;
             l += rs;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars.p_full[x]);
         }
-        mbar_arrive(&bars.kv_empty[s]);
+        mbar_arrive(&bars.desc_empty[di]);
         if (last) break;
     }
 
@@ -702,23 +836,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::bar_off);
-    Bars bars{bar + 0, bar + 1, bar + 3, bar + 5, bar + 7, bar + 9, bar + 11};
+    Bars bars{bar + 0,  bar + 1,  bar + 5,  bar + 9,  bar + 11, bar + 13,
+              bar + 15, bar + 17, bar + 19, bar + 21, bar + 23};
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::misc_off);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::misc_off + 4);
     uint32_t* patmap = reinterpret_cast<uint32_t*>(sm + L::patmap_off);
 
-    const int n = p.heads.n;
-    const int T = p.n_super - 1 - (int)(blockIdx.x / n);  // longest (latest) tiles first
-    const int pos = (int)(blockIdx.x % n);
+    // Work order: KV head by KV head (the CTAs in flight then stream one head's K/V,
+    // which fits in L2), longest (latest) super tiles first within a head.
+    int gi = 0;
+    while (gi + 1 < p.ngroups && (int)blockIdx.x >= (int)p.grp_start[gi + 1] * p.n_super) ++gi;
+    const int gsize = p.grp_start[gi + 1] - p.grp_start[gi];
+    const int rem = (int)blockIdx.x - (int)p.grp_start[gi] * p.n_super;
+    const int T = p.n_super - 1 - rem / gsize;
+    const int pos = p.grp_start[gi] + rem % gsize;
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
         // one read for the whole CTA: every thread must take the same branch
         *abort = *reinterpret_cast<volatile unsigned int*>(&g_abort_seq) == p.seq ? 1 : 0;
         mbar_init(bars.q_full, 1);
+        for (int i = 0; i < L::kDescRing; ++i) {
+            mbar_init(&bars.desc_full[i], 1);
+            mbar_init(&bars.desc_empty[i], 1 + kSoftmaxThreads);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars.kv_full[s], 1);
-            mbar_init(&bars.kv_empty[s], 1 + kSoftmaxThreads);
+            mbar_init(&bars.k_full[s], 1);
+            mbar_init(&bars.k_empty[s], 1);
+            mbar_init(&bars.v_full[s], 1);
+            mbar_init(&bars.v_empty[s], 1);
             mbar_init(&bars.s_full[s], 1);
             mbar_init(&bars.p_full[s], 128);
             mbar_init(&bars.o_done[s], 1);
@@ -745,8 +891,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == kProducerWarp) {
             run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
         } else if (warp == kMmaWarp) {
-            if ((threadIdx.x & 31) == 0) run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
-            __syncwarp();
+            run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
             tc_fence_before();
         }
     }
@@ -895,7 +1040,16 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
     p.sink = a.sink;
     p.window = a.window;
     p.err = a.err_count;
-    p.heads = a.heads;
+    // heads sorted by KV head (stable); each entry keeps its own per-pattern position
+    p.heads.n = 0;
+    p.ngroups = 0;
+    for (int g = 0; g < a.Hkv; ++g) {
+        const int start = p.heads.n;
+        for (int i = 0; i < a.heads.n; ++i)
+            if (kv_head_of(head_qh(a.heads.e[i]), a.Hq, a.Hkv) == g) p.heads.e[p.heads.n++] = a.heads.e[i];
+        if (p.heads.n > start) p.grp_start[p.ngroups++] = (uint16_t)start;
+    }
+    p.grp_start[p.ngroups] = (uint16_t)p.heads.n;
     const int patmap_words = p.nBw > p.nB / 8 + 1 ? p.nBw : p.nB / 8 + 1;
     const size_t smem = L::bytes(patmap_words);
     cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>,
