@@ -8,28 +8,26 @@
 // slash diagonals touch (Vertical-Slash), without counting a key twice.
 //
 // Work item = one query head x one 256-row "super tile" (four 64-row query
-// blocks).  The CTA holds the super tile as two 128-row slots that share
-// every key group brought into shared memory:
+// blocks), held as two 128-row slots.  The producer enumerates the item's
+// key chunks -- one 64-key block, or up to 64 gathered vertical columns --
+// each with a 4-bit mask (one bit per query block); a chunk is computed for
+// the slots whose bits it carries, and rows whose bit is clear see -inf.
 //   warps 0-3  softmax, slot 0 (TMEM lanes 0-127 = rows 0-127)
 //   warps 4-7  softmax, slot 1 (rows 128-255)
-//   warp 8     producer: enumerates the key groups of the item and loads
-//              them (TMA for pairs of 64-key blocks, cp.async gathers for
-//              vertical columns), two stages deep
-//   warp 9     MMA issuer: S = Q K^T (SS form) and O += P V (TS form, P read
-//              from TMEM), FA-style ping-pong between the two slots.
-// A key group is 128 keys: two (not necessarily adjacent) 64-key blocks, or
-// up to 128 gathered columns.  Each block / column carries a 4-bit mask, one
-// bit per query block, so one group serves rows with different masks; rows
-// whose bit is clear see -inf.  Only the diagonal block of a row, the edges
-// of an A-shape band and gathered columns need element-level tests.
+//   warp 8     producer: chunk list + TMA loads (cp.async gathers), 4 deep
+//   warps 9-10 MMA issuers, one per slot: S = Q K^T (SS form), O += P V (TS form)
+// Each slot double-buffers S in TMEM, so the tensor core computes S(n+1)
+// while the softmax works on S(n); O += P(n) V(n) follows once P(n) is
+// ready.  A slot's softmax therefore runs back to back, whether or not the
+// other slot needs the same chunk.
 //
-// TMEM (512 columns): slot x uses S at [256x, 256x+128) (P, bf16 pairs,
-// aliases its first 64 columns) and O at [256x+128, 256x+128+d).
+// TMEM (512 columns): slot x owns [256x, 256x+256): S buffers 0 and 1 at
+// +0 and +64 (64 columns each; P, bf16 pairs, reuses the first 32), O at
+// +128 (d columns).
 #include <cfloat>
 #include <cstring>
 #include <cudaTypedefs.h>
 
-#include "exp2_poly.h"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -38,34 +36,38 @@ namespace minfer {
 namespace {
 
 // 3 warpgroups: two softmax warpgroups (one per 128-row slot) and one for the
-// producer warp, the MMA warp and two idle warps.  Launched at 168 registers
+// producer warp, the two MMA warps and one idle warp.  Launched at 168 registers
 // per thread (65536 / 384, rounded down to 8); the softmax warpgroups then
-// take 224 and the third gives back down to 56: 2*128*224 + 128*56 = 384*168.
+// take 208 and the third 88: 2*128*208 + 128*88 = 384*168.
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+constexpr int kMmaWarp = 9;  // and 10: one MMA warp per slot
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168,
               "register split exceeds the launch budget");
 constexpr int kSoftmaxThreads = 256;
-constexpr int kGroupKeys = 128;
-constexpr int kPanelBytes = 128 * 128;  // 128 rows x one 64-column (128-byte) panel
+constexpr int kChunkKeys = 64;            // keys per chunk (one 64-key block)
+constexpr int kStages = 4;                // K and V ring depth (chunks)
+constexpr int kDescRing = 8;              // chunk descriptors in flight
+constexpr int kQPanel = 128 * 128;        // 128 rows x one 64-column (128-byte) panel
+constexpr int kKVPanel = kChunkKeys * 128;  // 64 rows x one panel
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by >8
 
-enum : int { kGrpNone = 0, kGrpTiles = 1, kGrpGather = 2 };
+enum : int { kChunkNone = 0, kChunkBlock = 1, kChunkGather = 2 };
 
-struct GroupDesc {
+struct ChunkDesc {
+    int info;  // type | need << 4 | last << 8: what the MMA issuer reads, in one load
     int type, last, need, ncols;
-    int b0, b1, m0, m1;
-    int cols[kGroupKeys];
-    uint8_t cm[kGroupKeys];
+    int b, m;  // block chunks: key block and its 4-bit query-block mask
+    int cols[kChunkKeys];
+    uint8_t cm[kChunkKeys];
 };
 
 struct GatherHeld {
-    int cols[kGroupKeys];
-    uint8_t cm[kGroupKeys];
+    int cols[kChunkKeys];
+    uint8_t cm[kChunkKeys];
 };
 
 // Sequence number of the last launch in which a CTA gave up waiting; later
@@ -73,7 +75,7 @@ struct GatherHeld {
 __device__ unsigned int g_abort_seq = 0;
 
 // First wait that gave up since the record was last read:
-// {launch seq, site, block, thread, group, parity, 0, 0}; site 0 = none.
+// {launch seq, site, block, thread, chunk, parity, 0, 0}; site 0 = none.
 __device__ int g_wait_fail[8];
 
 enum : int {
@@ -122,16 +124,15 @@ struct AttnParams {
 
 template <int D>
 struct Layout {
-    static constexpr int kQBytes = 128 * D * 2;   // one slot of Q
-    static constexpr int kKVBytes = kGroupKeys * D * 2;
+    static constexpr int kQBytes = 128 * D * 2;          // one slot of Q
+    static constexpr int kKVBytes = kChunkKeys * D * 2;  // one K or V stage
     static constexpr int q_off = 0;
     static constexpr int k_off = q_off + 2 * kQBytes;
-    static constexpr int v_off = k_off + 2 * kKVBytes;
-    static constexpr int kDescRing = 4;  // group descriptors in flight
-    static constexpr int desc_off = v_off + 2 * kKVBytes;
-    static constexpr int held_off = desc_off + kDescRing * (int)sizeof(GroupDesc);
+    static constexpr int v_off = k_off + kStages * kKVBytes;
+    static constexpr int desc_off = v_off + kStages * kKVBytes;
+    static constexpr int held_off = desc_off + kDescRing * (int)sizeof(ChunkDesc);
     static constexpr int bar_off = (held_off + (int)sizeof(GatherHeld) + 15) & ~15;
-    static constexpr int kNumBars = 24;
+    static constexpr int kNumBars = 1 + 2 * kDescRing + 3 * kStages + 12 + 2;
     static constexpr int misc_off = bar_off + kNumBars * 8;
     static constexpr int patmap_off = misc_off + 16;
     static size_t bytes(int patmap_words) {
@@ -142,22 +143,25 @@ struct Layout {
     }
 };
 
-// Pipeline barriers.  Group g (in publication order) uses descriptor slot
-// g % 4 and, if it carries keys, K stage and V stage g % 2.  K is released as
-// soon as the S = Q K^T of its group has run, V only after P V, so the next
-// K tile streams in while the current P V is still pending.
+// Pipeline barriers.  Chunk g (in publication order) uses descriptor slot
+// g % 8 and K/V stage g % 4.  kv_full completes once both tiles have landed
+// (the end marker completes it without data); since the producer writes a
+// chunk's descriptor before it arms kv_full, the MMA issuer needs only that
+// barrier.  K is released once the S of the chunk has run, V once every P V
+// that reads it has run.
+// Slot x's n-th chunk uses S buffer n % 2: s_full / p_full / pv_done are
+// per slot and per buffer, so no waiter can ever be lapped by two phases.
 struct Bars {
     uint64_t* q_full;
-    uint64_t* desc_full;   // [4] producer -> MMA, softmax
-    uint64_t* desc_empty;  // [4] MMA + 256 softmax threads -> producer
-    uint64_t* k_full;      // [2] TMA / gather -> MMA
-    uint64_t* k_empty;     // [2] MMA (after S) -> producer
-    uint64_t* v_full;      // [2]
-    uint64_t* v_empty;     // [2] MMA (after P V) -> producer
-    uint64_t* s_full;      // [2] per slot: S ready in TMEM
-    uint64_t* p_full;      // [2] per slot: P written to TMEM
-    uint64_t* o_done;      // [2] per slot: last P V done
-    uint64_t* drain;
+    uint64_t* desc_full;   // [8] producer -> MMA, softmax
+    uint64_t* desc_empty;  // [8] MMA + 256 softmax threads -> producer
+    uint64_t* kv_full;     // [4] TMA / gather -> MMA
+    uint64_t* k_empty;     // [4] MMA (after S) -> producer
+    uint64_t* v_empty;     // [4] MMA (after P V) -> producer
+    uint64_t* s_full;      // [2 slots][2 buffers] S ready in TMEM
+    uint64_t* p_full;      // [2][2] P written to TMEM (128 softmax threads)
+    uint64_t* pv_done;     // [2][2] O += P V of that buffer has run
+    uint64_t* drain;       // [2] per MMA warp: all its MMAs have run
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -191,26 +195,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// 2^x for a pair on the FMA pipe (method and error bound in exp2_poly.h).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    const uint64_t xc = f2_pack(fmaxf(x0, kExp2Clamp), fmaxf(x1, kExp2Clamp));
-    const uint64_t t = f2_add(xc, f2_pack(kExp2Round, kExp2Round));        // round to nearest
-    const uint64_t n = f2_add(t, f2_pack(-kExp2Round, -kExp2Round));       // n as float
-    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);                 // x - n, exact
-    uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
-    q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
-    float q0, q1, t0, t1;
-    f2_unpack(q, q0, q1);
-    f2_unpack(t, t0, t1);
-    // n sits in the low mantissa bits of t; (bits(t) << 23) adds n to the exponent
-    const float r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    const float r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-    return f2_pack(r0, r1);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -232,12 +216,11 @@ struct Producer {
     uint8_t* sm;
     Bars bars;
     volatile int* abort;
-    GroupDesc* desc;
+    ChunkDesc* desc;
     GatherHeld* held;
     int g;        // KV head
     int pub = 0;  // descriptors published
-    int nk = 0;   // K stages filled
-    int nv = 0;   // V stages filled
+    int nkv = 0;  // K/V stages armed (one per descriptor)
     int lane;
     bool ok = true;
 
@@ -255,78 +238,66 @@ struct Producer {
         }
         return w;
     }
-    __device__ GroupDesc* acquire_desc() {
-        const int i = pub & (L::kDescRing - 1);
-        if (pub >= L::kDescRing && !wait(&bars.desc_empty[i], ((pub / L::kDescRing) - 1) & 1, pub))
+    __device__ ChunkDesc* acquire_desc() {
+        const int i = pub % kDescRing;
+        if (pub >= kDescRing && !wait(&bars.desc_empty[i], ((pub / kDescRing) - 1) & 1, pub))
             return nullptr;
         return &desc[i];
     }
     __device__ void publish_desc() {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.desc_full[pub & (L::kDescRing - 1)]);
+        if (lane == 0) mbar_arrive(&bars.desc_full[pub % kDescRing]);
         ++pub;
     }
-    __device__ bool acquire_k(int& s) {
-        s = nk & 1;
-        return nk < 2 || wait(&bars.k_empty[s], ((nk >> 1) - 1) & 1, nk);
-    }
-    __device__ bool acquire_v(int& s) {
-        s = nv & 1;
-        return nv < 2 || wait(&bars.v_empty[s], ((nv >> 1) - 1) & 1, nv);
+    // the stage of the next descriptor, once its previous K and V are released
+    __device__ bool acquire_kv(int& s) {
+        s = nkv % kStages;
+        if (nkv < kStages) return true;
+        const int par = ((nkv / kStages) - 1) & 1;
+        return wait(&bars.k_empty[s], par, nkv) && wait(&bars.v_empty[s], par, nkv);
     }
 
-    __device__ void tiles(int b0, int m0, int b1, int m1) {
+    // one 64-key block with its query-block mask
+    __device__ void block(int b, int m) {
         if (!ok) return;
-        GroupDesc* d = acquire_desc();
+        ChunkDesc* d = acquire_desc();
         if (!d) return;
         if (lane == 0) {
-            d->type = kGrpTiles;
+            const int need = ((m & 0x3) ? 1 : 0) | ((m & 0xC) ? 2 : 0);
+            d->info = kChunkBlock | (need << 4);
+            d->type = kChunkBlock;
             d->last = 0;
-            d->need = (((m0 | m1) & 0x3) ? 1 : 0) | (((m0 | m1) & 0xC) ? 2 : 0);
+            d->need = need;
             d->ncols = 0;
-            d->b0 = b0;
-            d->b1 = b1;
-            d->m0 = m0;
-            d->m1 = m1;
+            d->b = b;
+            d->m = m;
         }
         publish_desc();
-        const int row0 = g * p.N + 64 * b0, row1 = g * p.N + 64 * b1;
-        int sk;
-        if (!acquire_k(sk)) return;
+        int st;
+        if (!acquire_kv(st)) return;
         if (lane == 0) {
-            mbar_arrive_expect_tx(&bars.k_full[sk], L::kKVBytes);
-            uint8_t* kd = sm + L::k_off + sk * L::kKVBytes;
+            const int row = g * p.N + kChunkKeys * b;
+            mbar_arrive_expect_tx(&bars.kv_full[st], 2 * L::kKVBytes);
+            uint8_t* kd = sm + L::k_off + st * L::kKVBytes;
+            uint8_t* vd = sm + L::v_off + st * L::kKVBytes;
 #pragma unroll
-            for (int pn = 0; pn < D / 64; ++pn) {
-                tma_load_2d(kd + pn * kPanelBytes, tmK, 64 * pn, row0, &bars.k_full[sk]);
-                tma_load_2d(kd + pn * kPanelBytes + kPanelBytes / 2, tmK, 64 * pn, row1,
-                            &bars.k_full[sk]);
-            }
+            for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_2d(kd + pn * kKVPanel, tmK, 64 * pn, row, &bars.kv_full[st]);
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_2d(vd + pn * kKVPanel, tmV, 64 * pn, row, &bars.kv_full[st]);
         }
         __syncwarp();
-        ++nk;
-        int sv;
-        if (!acquire_v(sv)) return;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&bars.v_full[sv], L::kKVBytes);
-            uint8_t* vd = sm + L::v_off + sv * L::kKVBytes;
-#pragma unroll
-            for (int pn = 0; pn < D / 64; ++pn) {
-                tma_load_2d(vd + pn * kPanelBytes, tmV, 64 * pn, row0, &bars.v_full[sv]);
-                tma_load_2d(vd + pn * kPanelBytes + kPanelBytes / 2, tmV, 64 * pn, row1,
-                            &bars.v_full[sv]);
-            }
-        }
-        __syncwarp();
-        ++nv;
+        ++nkv;
     }
 
+    // up to 64 gathered columns
     __device__ void gather(int n) {
         if (!ok) return;
-        GroupDesc* d = acquire_desc();
+        ChunkDesc* d = acquire_desc();
         if (!d) return;
         int need = 0;
-        for (int c = lane; c < kGroupKeys; c += 32) {
+        for (int c = lane; c < kChunkKeys; c += 32) {
             const bool v = c < n;
             const int col = v ? held->cols[c] : held->cols[0];
             const int cm = v ? held->cm[c] : 0;
@@ -336,60 +307,63 @@ struct Producer {
         }
         for (int off = 16; off >= 1; off >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, off);
         if (lane == 0) {
-            d->type = kGrpGather;
+            const int nd = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
+            d->info = kChunkGather | (nd << 4);
+            d->type = kChunkGather;
             d->last = 0;
-            d->need = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
+            d->need = nd;
             d->ncols = n;
-            d->b0 = d->b1 = -1;
-            d->m0 = d->m1 = 0;
+            d->b = -1;
+            d->m = 0;
         }
         publish_desc();
-        int sk, sv;
-        if (!acquire_k(sk) || !acquire_v(sv)) return;
-        uint8_t* kd = sm + L::k_off + sk * L::kKVBytes;
-        uint8_t* vd = sm + L::v_off + sv * L::kKVBytes;
+        int st;
+        if (!acquire_kv(st)) return;
+        uint8_t* kd = sm + L::k_off + st * L::kKVBytes;
+        uint8_t* vd = sm + L::v_off + st * L::kKVBytes;
         constexpr int kChunks = D / 8;  // 16-byte chunks per row
         const bf16* kb = p.k + (size_t)g * p.N * D;
         const bf16* vb = p.v + (size_t)g * p.N * D;
-        for (int idx = lane; idx < kGroupKeys * kChunks; idx += 32) {
+        for (int idx = lane; idx < kChunkKeys * kChunks; idx += 32) {
             const int r = idx / kChunks, c = idx % kChunks;
             const size_t src = (size_t)d->cols[r] * D + c * 8;
-            const int dst = (c >> 3) * kPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+            const int dst = (c >> 3) * kKVPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4);
             cp_async_16(kd + dst, kb + src);
             cp_async_16(vd + dst, vb + src);
         }
         cp_async_wait_all();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&bars.k_full[sk]);
-            mbar_arrive(&bars.v_full[sv]);
-        }
-        ++nk;
-        ++nv;
+        if (lane == 0) mbar_arrive(&bars.kv_full[st]);
+        ++nkv;
     }
 
+    // end marker: a descriptor with no keys, signalled through kv_full like the rest
     __device__ void finish() {
         if (!ok) return;
-        GroupDesc* d = acquire_desc();
+        ChunkDesc* d = acquire_desc();
         if (!d) return;
         if (lane == 0) {
-            d->type = kGrpNone;
+            d->info = kChunkNone | (1 << 8);
+            d->type = kChunkNone;
             d->last = 1;
             d->need = 0;
             d->ncols = 0;
         }
         publish_desc();
+        int st;
+        if (!acquire_kv(st)) return;
+        if (lane == 0) mbar_arrive(&bars.kv_full[st]);
+        __syncwarp();
+        ++nkv;
     }
 
     // Wait (bounded) until every copy this warp started has landed, so that
     // no TMA write can reach shared memory after the CTA exits.
     __device__ void drain() {
         if (lane != 0) return;
-        for (int u = nk - 2; u < nk; ++u)
-            if (u >= 0) mbar_wait_budget(&bars.k_full[u & 1], (u >> 1) & 1);
-        for (int u = nv - 2; u < nv; ++u)
-            if (u >= 0) mbar_wait_budget(&bars.v_full[u & 1], (u >> 1) & 1);
+        for (int u = nkv - kStages; u < nkv; ++u)
+            if (u >= 0) mbar_wait_budget(&bars.kv_full[u % kStages], (u / kStages) & 1);
     }
 };
 
@@ -417,7 +391,7 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
         mbar_arrive_expect_tx(bars.q_full, 2 * L::kQBytes);
         for (int x = 0; x < 2; ++x)
             for (int pn = 0; pn < D / 64; ++pn)
-                tma_load_2d(sm + L::q_off + x * L::kQBytes + pn * kPanelBytes, tmQ, 64 * pn,
+                tma_load_2d(sm + L::q_off + x * L::kQBytes + pn * kQPanel, tmQ, 64 * pn,
                             qh * p.N + 256 * T + 128 * x, bars.q_full);
     }
 
@@ -447,12 +421,11 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
     __syncwarp();
 
     Producer<D> pr{p, tmK, tmV, sm, bars, abort,
-                   reinterpret_cast<GroupDesc*>(sm + L::desc_off),
+                   reinterpret_cast<ChunkDesc*>(sm + L::desc_off),
                    reinterpret_cast<GatherHeld*>(sm + L::held_off), g};
     pr.lane = lane;
 
-    // --- 64-key blocks, ascending, paired into 128-key groups
-    int pend_b = -1, pend_m = 0;
+    // --- 64-key blocks, ascending, one chunk each
     for (int base = 0; base <= bmax && pr.ok; base += 32) {
         const int b = base + lane;
         int m = 0;
@@ -477,18 +450,11 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
             const int src = __ffs(bal) - 1;
             bal &= bal - 1;
             const int mm = __shfl_sync(0xffffffffu, m, src);
-            if (pend_b < 0) {
-                pend_b = base + src;
-                pend_m = mm;
-            } else {
-                pr.tiles(pend_b, pend_m, base + src, mm);
-                pend_b = -1;
-            }
+            pr.block(base + src, mm);
         }
     }
-    if (pend_b >= 0) pr.tiles(pend_b, pend_m, pend_b, 0);
 
-    // --- Vertical-Slash: gathered columns not already inside a computed tile
+    // --- Vertical-Slash: gathered columns not already inside a computed block
     if (pattern == MI_PATTERN_VS && pr.ok) {
         const int vc = p.vcnt[pidx];
         const int32_t* vl = p.vlist + (size_t)pidx * p.vcap;
@@ -511,14 +477,14 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
             const unsigned bal = __ballot_sync(0xffffffffu, m != 0);
             const int rank = __popc(bal & ((1u << lane) - 1u));
             const int navail = __popc(bal);
-            const int take = min(navail, kGroupKeys - n_held);
+            const int take = min(navail, kChunkKeys - n_held);
             if (m && rank < take) {
                 held->cols[n_held + rank] = j;
                 held->cm[n_held + rank] = (uint8_t)m;
             }
             __syncwarp();
             n_held += take;
-            if (n_held == kGroupKeys) {
+            if (n_held == kChunkKeys) {
                 pr.gather(n_held);
                 n_held = 0;
                 if (m && rank >= take) {
@@ -539,108 +505,143 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
     pr.drain();
 }
 
-// ------------------------------------------------------------- MMA issuer
-// The whole warp runs this loop converged: bookkeeping and descriptors are
-// uniform, lane 0 alone polls the barriers and broadcasts the outcome, and
-// elect.sync inside the issue instructions picks the single issuing lane.
+// ------------------------------------------------------------- MMA issuers
+// One MMA warp per slot (warp 9 for rows 0-127, warp 10 for rows 128-255):
+// each issues only its own slot's S and P V, so the two warps' bookkeeping
+// overlaps the other's MMAs in the tensor pipe.  They share the K/V stages
+// and the descriptors, which are released once both have passed a chunk
+// (k_empty, v_empty and the MMA share of desc_empty count two arrivals; a
+// warp can see chunk g+4's K/V only after both released chunk g, so no
+// arrival can fall into the wrong phase).
+//
+// The warp runs its loop converged, with every MMA operand derived from
+// lane-0 broadcasts and ballots, so the compiler keeps the operands in
+// uniform registers (one it cannot prove uniform is moved there on every
+// issue, which is slower than the tensor pipe); elect.sync inside the issue
+// instructions picks the issuing lane.  An mbarrier probe costs about 200
+// cycles even on a completed phase, so each round probes, in one
+// non-blocking test_wait, the next chunk's K/V (lane 0; once seen it stays
+// landed until used) and the P of the slot's oldest chunk still waiting for
+// O += P V (lane 1), and then issues what is ready:
+//   O += P V for that chunk, then
+//   S = Q K^T of the next chunk (if the slot needs it) into the slot's other
+//   S buffer, once at most one chunk waits for P V (the buffer S overwrites
+//   holds the P of the chunk before last, which its P V must have read
+//   first; one thread's MMAs run in issue order).
+// So the tensor core computes S(n+1) while the softmax works on S(n).
 template <int D>
 __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int32_t* err,
-                        unsigned int seq, uint32_t tmem) {
+                        unsigned int seq, uint32_t tmem, int x) {
     using L = Layout<D>;
     const int lane = threadIdx.x & 31;
-    const uint32_t idS = idesc_bf16_f32(128, kGroupKeys, false);
+    const uint32_t idS = idesc_bf16_f32(128, kChunkKeys, false);
     const uint32_t idO = idesc_bf16_f32(128, D, true);
-    const uint32_t q_addr = smem_u32(sm + L::q_off);
-    const uint32_t k_addr = smem_u32(sm + L::k_off);
-    const uint32_t v_addr = smem_u32(sm + L::v_off);
-    const GroupDesc* desc = reinterpret_cast<const GroupDesc*>(sm + L::desc_off);
-    auto wait = [&](uint64_t* bar, int parity) -> bool {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(bar, parity, abort);
-        return __shfl_sync(0xffffffffu, w, 0);
-    };
+    tmem = __shfl_sync(0xffffffffu, tmem, 0);
+    x = __shfl_sync(0xffffffffu, x, 0);
+    const uint32_t tSlot = tmem + 256 * x;
+    const uint32_t q_addr = __shfl_sync(0xffffffffu, smem_u32(sm + L::q_off + x * L::kQBytes), 0);
+    const uint32_t k_addr = __shfl_sync(0xffffffffu, smem_u32(sm + L::k_off), 0);
+    const uint32_t v_addr = __shfl_sync(0xffffffffu, smem_u32(sm + L::v_off), 0);
+    const ChunkDesc* desc = reinterpret_cast<const ChunkDesc*>(sm + L::desc_off);
+    uint64_t* const p_full = bars.p_full + 2 * x;
+    uint64_t* const s_full = bars.s_full + 2 * x;
+    uint64_t* const pv_done = bars.pv_done + 2 * x;
 
-    int pend[2] = {-1, -1}, npv[2] = {0, 0}, np[2] = {0, 0};
-    int vuses[2] = {0, 0};
-    bool ok = wait(bars.q_full, 0);
-    if (!ok && lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, 0);
-    int g = 0;
-    while (ok) {
-        const int di = g & (L::kDescRing - 1);
-        if (!wait(&bars.desc_full[di], (g / L::kDescRing) & 1)) {
-            if (lane == 0 && !*abort)
-                record_wait_failure(seq, kSiteMmaFull, g, (g / L::kDescRing) & 1);
-            ok = false;
-            break;
+    bool ok = true;
+    {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(bars.q_full, 0, abort);
+        ok = __shfl_sync(0xffffffffu, w, 0);
+        if (!ok && lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, x);
+    }
+
+    int g = 0;              // next chunk to read
+    bool done = false;      // end marker read
+    bool kv_ready = false;  // chunk g's K/V seen landed
+    int nS = 0;             // S issued
+    int cnt = 0;            // chunks whose P V is still to issue (0..2)
+    int pc0 = 0, pc1 = 0;   // the oldest of them, the newer one
+    long long t_last = clock64();
+    while (ok && !(done && cnt == 0)) {
+        const bool want_kv = !done && !kv_ready;
+        uint64_t* pb = bars.q_full;  // completed: a harmless target for idle lanes
+        uint32_t par = 0;
+        bool live = false;
+        if (lane == 0 && want_kv) {
+            pb = &bars.kv_full[g % kStages];
+            par = (g / kStages) & 1;
+            live = true;
+        } else if (lane == 1 && cnt > 0) {
+            const int sidx = nS - cnt;
+            pb = &p_full[sidx & 1];
+            par = (sidx >> 1) & 1;
+            live = true;
         }
-        const int type = desc[di].type, need = desc[di].need, last = desc[di].last;
-        const int s = g & 1;  // data groups are numbered like descriptors (the end marker is last)
-        bool k_ready = false;
-        // per slot: first the pending O += P V (needs only P and V), then S of
-        // this group (needs K): a late K tile does not hold back the other work
-        for (int x = 0; x < 2 && ok; ++x) {
-            if (pend[x] >= 0) {
-                // P of the slot's previous group, then its V: issue O += P V
-                const int pg = pend[x], st = pg & 1;
-                if (!wait(&bars.p_full[x], np[x] & 1) || !wait(&bars.v_full[st], (pg >> 1) & 1)) {
-                    if (lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaP, g, np[x] & 1);
-                    ok = false;
-                    break;
-                }
-                ++np[x];
-                tc_fence_after();
-                const uint32_t tP = tmem + 256 * x;
-                const uint32_t tO = tmem + 256 * x + 128;
-#pragma unroll
-                for (int kk = 0; kk < kGroupKeys / 16; ++kk) {
-                    const uint64_t bdesc =
-                        sw128_desc(v_addr + st * L::kKVBytes + kk * 2048, kPanelBytes, 1024);
-                    mma_ts_warp(tO, tP + kk * 8, bdesc, idO, (npv[x] > 0 || kk > 0) ? 1u : 0u);
-                }
-                ++npv[x];
-                if (--vuses[st] == 0) mma_commit_warp(&bars.v_empty[st]);
-                pend[x] = -1;
+        const bool hit = mbar_test_wait(pb, par) && live;
+        const unsigned bal = __ballot_sync(0xffffffffu, hit);
+        kv_ready |= (bal & 1u) != 0;
+        const bool hp = (bal >> 1) & 1u;
+        const bool can_s = kv_ready && cnt - (hp ? 1 : 0) <= 1;
+        if (!(hp || can_s)) {
+            const bool give_up = *abort || clock64() - t_last > kWaitBudgetCycles;
+            if (__any_sync(0xffffffffu, give_up)) {
+                if (lane == 0 && !*abort)
+                    record_wait_failure(seq, want_kv ? kSiteMmaFull : kSiteMmaP, g, cnt | x << 4);
+                ok = false;
             }
-            if (type != kGrpNone && ((need >> x) & 1)) {
-                if (!k_ready) {
-                    if (!wait(&bars.k_full[s], (g >> 1) & 1)) {
-                        if (lane == 0 && !*abort)
-                            record_wait_failure(seq, kSiteMmaFull, g, (g >> 1) & 1);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    k_ready = true;
-                }
-                const uint32_t tS = tmem + 256 * x;
+            continue;
+        }
+        t_last = clock64();
+        tc_fence_after();
+        if (hp) {  // O += P V for the oldest pending chunk
+            const int sidx = nS - cnt, st = pc0 % kStages;
+            const uint32_t tP = tSlot + 64 * (sidx & 1);
+#pragma unroll
+            for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
+                const uint64_t bdesc =
+                    sw128_desc(v_addr + st * L::kKVBytes + kk * 2048, kKVPanel, 1024);
+                mma_ts_warp(tSlot + 128, tP + kk * 8, bdesc, idO, (sidx > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_warp(&pv_done[sidx & 1]);
+            mma_commit_warp(&bars.v_empty[st]);  // this slot is done with the V stage
+            pc0 = pc1;
+            --cnt;
+        }
+        if (can_s) {  // the next chunk (its descriptor was written before kv_full was armed)
+            kv_ready = false;
+            const int di = g % kDescRing, s = g % kStages;
+            const int info = __shfl_sync(0xffffffffu, desc[di].info, 0);
+            const int type = info & 0xF, last = (info >> 8) & 1;
+            if ((info >> (4 + x)) & 1) {
+                const uint32_t tS = tSlot + 64 * (nS & 1);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int pn = kk >> 2, off = (kk & 3) * 32;
-                    const uint64_t adesc =
-                        sw128_desc(q_addr + x * L::kQBytes + pn * kPanelBytes + off, 16, 1024);
+                    const uint64_t adesc = sw128_desc(q_addr + pn * kQPanel + off, 16, 1024);
                     const uint64_t bdesc =
-                        sw128_desc(k_addr + s * L::kKVBytes + pn * kPanelBytes + off, 16, 1024);
+                        sw128_desc(k_addr + s * L::kKVBytes + pn * kKVPanel + off, 16, 1024);
                     mma_ss_warp(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit_warp(&bars.s_full[x]);
-                pend[x] = g;
+                mma_commit_warp(&s_full[nS & 1]);
+                mma_commit_warp(&bars.k_empty[s]);  // K free once both slots' S have run
+                if (cnt == 0) pc0 = g;
+                else pc1 = g;
+                ++cnt;
+                ++nS;
+            } else if (type != kChunkNone) {
+                // this slot skips the chunk: release its share of the stage now
+                mbar_arrive_warp(&bars.k_empty[s]);
+                mbar_arrive_warp(&bars.v_empty[s]);
             }
+            mbar_arrive_warp(&bars.desc_empty[di]);
+            if (last) done = true;
+            else ++g;
         }
-        if (!ok) break;
-        if (type != kGrpNone) {
-            mma_commit_warp(&bars.k_empty[s]);  // K free once this group's S has run
-            vuses[s] = __popc(need);
-        }
-        mbar_arrive_warp(&bars.desc_empty[di]);
-        if (last) break;
-        ++g;
     }
     if (!ok && lane == 0) set_abort(abort, err, seq);
-    for (int x = 0; x < 2; ++x)
-        if (npv[x] > 0) mma_commit_warp(&bars.o_done[x]);
-    // every MMA must have finished before TMEM is released
-    mma_commit_warp(bars.drain);
-    if (lane == 0) mbar_wait_budget(bars.drain, 0);
+    // every MMA of this warp must have finished before TMEM is released
+    mma_commit_warp(&bars.drain[x]);
+    if (lane == 0) mbar_wait_budget(&bars.drain[x], 0);
     __syncwarp();
 }
 
@@ -659,85 +660,92 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     const int qh = head_qh(e), pattern = head_pattern(e);
     const bool ashape = pattern == MI_PATTERN_ASHAPE;
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    const uint32_t tS = tmem + 256 * x + lane_off;
-    const uint32_t tO = tmem + 256 * x + 128 + lane_off;
-    const GroupDesc* desc = reinterpret_cast<const GroupDesc*>(sm + L::desc_off);
+    // warp-uniform TMEM address (tcgen05.ld/st take it from a uniform register)
+    const uint32_t tSlot = __shfl_sync(0xffffffffu, tmem + 256 * x + lane_off, 0);
+    const uint32_t tO = tSlot + 128;
+    const ChunkDesc* desc = reinterpret_cast<const ChunkDesc*>(sm + L::desc_off);
+    const float cs = p.scale_log2;
 
     float m = -INFINITY, l = 0.f;
-    int ns = 0;
+    int n = 0;  // chunks this slot has processed
     bool ok = true;
     for (int g = 0;; ++g) {
-        const int di = g & (L::kDescRing - 1);
-        const int dpar = (g / L::kDescRing) & 1;
+        const int di = g % kDescRing;
+        const int dpar = (g / kDescRing) & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.desc_full[di], dpar, abort))) {
             if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxFull, g, dpar);
             ok = false;
             break;
         }
-        const GroupDesc& d = desc[di];
+        const ChunkDesc& d = desc[di];
         const int type = d.type, last = d.last;
-        if (type != kGrpNone && ((d.need >> x) & 1)) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[x], ns & 1, abort))) {
-                if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxS, g, ns & 1);
+        if (type != kChunkNone && ((d.need >> x) & 1)) {
+            const int b = n & 1;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&bars.s_full[2 * x + b], (n >> 1) & 1, abort))) {
+                if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxS, g, (n >> 1) & 1);
                 ok = false;
                 break;
             }
-            ++ns;
             tc_fence_after();
-            float v[kGroupKeys];
+            const uint32_t tS = __shfl_sync(0xffffffffu, tSlot + 64 * b, 0);
+            float v[kChunkKeys];
             {
-                uint32_t r[kGroupKeys];
-                tmem_ld128(tS, r);  // the whole row of S: one TMEM round trip
+                uint32_t r[32];
+                tmem_ld32(tS, r);
 #pragma unroll
-                for (int u = 0; u < kGroupKeys; ++u) v[u] = __uint_as_float(r[u]);
+                for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(r[u]);
+                tmem_ld32(tS + 32, r);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[32 + u] = __uint_as_float(r[u]);
             }
-            if (type == kGrpTiles) {
+            if (type == kChunkBlock) {
+                const int bit = (d.m >> qi) & 1;
+                const long long j0 = 64LL * d.b;
+                const bool full = bit && (j0 + 63 <= i) &&
+                                  (!ashape || j0 + 63 < p.sink || i - j0 < p.window);
+                if (!full) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int b = h ? d.b1 : d.b0;
-                    const int bit = ((h ? d.m1 : d.m0) >> qi) & 1;
-                    const long long j0 = 64LL * b;
-                    const bool full = bit && (j0 + 63 <= i) &&
-                                      (!ashape || j0 + 63 < p.sink || i - j0 < p.window);
-                    if (!full) {
-#pragma unroll
-                        for (int c = 0; c < 64; ++c) {
-                            const long long j = j0 + c;
-                            const bool keep = bit && j <= i &&
-                                              (!ashape || j < p.sink || i - j < p.window);
-                            if (!keep) v[64 * h + c] = -INFINITY;
-                        }
+                    for (int c = 0; c < kChunkKeys; ++c) {
+                        const long long j = j0 + c;
+                        const bool keep =
+                            bit && j <= i && (!ashape || j < p.sink || i - j < p.window);
+                        if (!keep) v[c] = -INFINITY;
                     }
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < kGroupKeys; ++c) {
+                for (int c = 0; c < kChunkKeys; ++c) {
                     const bool keep = ((d.cm[c] >> qi) & 1) && (long long)d.cols[c] <= i;
                     if (!keep) v[c] = -INFINITY;
                 }
             }
             // raw scores: the scale (> 0) commutes with the max and is folded into
             // the exponent below (one packed FFMA per pair)
-            const float cs = p.scale_log2;
-            // four independent max chains (latency), then combined
-            float mq[4] = {fmaxf(v[0], v[1]), fmaxf(v[2], v[3]), fmaxf(v[4], v[5]),
-                           fmaxf(v[6], v[7])};
+            float mq[2] = {fmaxf(v[0], v[1]), fmaxf(v[2], v[3])};
 #pragma unroll
-            for (int c = 8; c < kGroupKeys; c += 8) {
-#pragma unroll
-                for (int w4 = 0; w4 < 4; ++w4)
-                    mq[w4] = fmax3(mq[w4], v[c + 2 * w4], v[c + 2 * w4 + 1]);
+            for (int c = 4; c < kChunkKeys; c += 4) {
+                mq[0] = fmax3(mq[0], v[c], v[c + 1]);
+                mq[1] = fmax3(mq[1], v[c + 2], v[c + 3]);
             }
-            float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
-            mx *= cs;
+            const float mx = fmaxf(mq[0], mq[1]) * cs;
             // Lazy rescale: a row moves its reference max only when the max grew by
-            // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  The
-            // TMEM accesses are .sync.aligned, so the whole warp takes the branch
+            // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  O may be
+            // rescaled only once the slot's previous O += P V has run.  The TMEM
+            // accesses are .sync.aligned, so the whole warp takes the branch
             // together; rows that do not need it scale by 1.
             const bool want = mx > m + kRescaleThreshold;
             if (__any_sync(0xffffffffu, want)) {
                 const float alpha = want ? ex2(m - mx) : 1.f;  // 0 while m is -inf
-                if (ns > 1) {
+                if (n > 0) {
+                    const int pb = (n - 1) & 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + pb],
+                                                           ((n - 1) >> 1) & 1, abort))) {
+                        if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxO, g, 0);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                     uint32_t o[32];
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -753,47 +761,41 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
             }
             const float mu = (m == -INFINITY) ? 0.f : m;
             const uint64_t cs2 = f2_pack(cs, cs), nmu2 = f2_pack(-mu, -mu);
-            // four independent packed row-sum accumulators (latency)
             uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f),
                                 f2_pack(0.f, 0.f)};
+            uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const uint64_t x2 =
-                        f2_fma(f2_pack(v[64 * c + 2 * u], v[64 * c + 2 * u + 1]), cs2, nmu2);
-                    // all exponentials on MUFU: measured faster than moving a share to
-                    // the FMA pipe, the softmax warp is bound by its own issue rate
-                    float x0, x1;
-                    f2_unpack(x2, x0, x1);
-                    const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
-                    sum2[u & 3] = f2_add(sum2[u & 3], p2);
-                    float p0, p1;
-                    f2_unpack(p2, p0, p1);
-                    pk[u] = pack_bf16(p0, p1);
-                }
-                tmem_st32(tS + 32 * c, pk);
+            for (int u = 0; u < 32; ++u) {
+                const uint64_t x2 = f2_fma(f2_pack(v[2 * u], v[2 * u + 1]), cs2, nmu2);
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+                sum2[u & 3] = f2_add(sum2[u & 3], p2);
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
+                pk[u] = pack_bf16(p0, p1);
             }
+            tmem_st32(tS, pk);  // P over the first 32 columns of its S buffer
             float s0, s1;
             f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
-            const float rs = s0 + s1;
-            l += rs;
+            l += s0 + s1;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars.p_full[x]);
+            mbar_arrive(&bars.p_full[2 * x + b]);
+            ++n;
         }
         mbar_arrive(&bars.desc_empty[di]);
         if (last) break;
     }
 
     // epilogue: O / l -> bf16, lse
-    bool have = ns > 0 && ok;
+    bool have = n > 0 && ok;
     if (have) {
-        have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[x], 0, abort));
+        have = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + ((n - 1) & 1)],
+                                                 ((n - 1) >> 1) & 1, abort));
         if (!have && !*abort) record_wait_failure(p.seq, kSiteSoftmaxO, -1, 0);
     }
-    if (!ok || (ns > 0 && !have)) set_abort(abort, p.err, p.seq);
+    if (!ok || (n > 0 && !have)) set_abort(abort, p.err, p.seq);
     tc_fence_after();
     const bool row_ok = i < p.N;
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -836,8 +838,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::bar_off);
-    Bars bars{bar + 0,  bar + 1,  bar + 5,  bar + 9,  bar + 11, bar + 13,
-              bar + 15, bar + 17, bar + 19, bar + 21, bar + 23};
+    Bars bars;
+    {
+        uint64_t* q = bar;
+        bars.q_full = q;
+        q += 1;
+        bars.desc_full = q;
+        q += kDescRing;
+        bars.desc_empty = q;
+        q += kDescRing;
+        bars.kv_full = q;
+        q += kStages;
+        bars.k_empty = q;
+        q += kStages;
+        bars.v_empty = q;
+        q += kStages;
+        bars.s_full = q;
+        q += 4;
+        bars.p_full = q;
+        q += 4;
+        bars.pv_done = q;
+        q += 4;
+        bars.drain = q;
+    }
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::misc_off);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::misc_off + 4);
     uint32_t* patmap = reinterpret_cast<uint32_t*>(sm + L::patmap_off);
@@ -856,20 +879,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one read for the whole CTA: every thread must take the same branch
         *abort = *reinterpret_cast<volatile unsigned int*>(&g_abort_seq) == p.seq ? 1 : 0;
         mbar_init(bars.q_full, 1);
-        for (int i = 0; i < L::kDescRing; ++i) {
-            mbar_init(&bars.desc_full[i], 1);
-            mbar_init(&bars.desc_empty[i], 1 + kSoftmaxThreads);
+        for (int k = 0; k < kDescRing; ++k) {
+            mbar_init(&bars.desc_full[k], 1);
+            mbar_init(&bars.desc_empty[k], 2 + kSoftmaxThreads);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars.k_full[s], 1);
-            mbar_init(&bars.k_empty[s], 1);
-            mbar_init(&bars.v_full[s], 1);
-            mbar_init(&bars.v_empty[s], 1);
-            mbar_init(&bars.s_full[s], 1);
-            mbar_init(&bars.p_full[s], 128);
-            mbar_init(&bars.o_done[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars.kv_full[s], 1);
+            mbar_init(&bars.k_empty[s], 2);  // one arrival per MMA warp
+            mbar_init(&bars.v_empty[s], 2);
         }
-        mbar_init(bars.drain, 1);
+        for (int k = 0; k < 4; ++k) {
+            mbar_init(&bars.s_full[k], 1);
+            mbar_init(&bars.p_full[k], 128);
+            mbar_init(&bars.pv_done[k], 1);
+        }
+        mbar_init(&bars.drain[0], 1);
+        mbar_init(&bars.drain[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -890,8 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_dec<kControlRegs>();
         if (warp == kProducerWarp) {
             run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
-        } else if (warp == kMmaWarp) {
-            run_mma<D>(sm, bars, abort, p.err, p.seq, tmem);
+        } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+            run_mma<D>(sm, bars, abort, p.err, p.seq, tmem, warp - kMmaWarp);
             tc_fence_before();
         }
     }
