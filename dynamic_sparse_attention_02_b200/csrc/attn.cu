@@ -561,6 +561,7 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
     int nS = 0;             // S issued
     int cnt = 0;            // chunks whose P V is still to issue (0..2)
     int pc0 = 0, pc1 = 0;   // the oldest of them, the newer one
+    unsigned idle = 0;      // rounds that found nothing to do
     long long t_last = clock64();
     while (ok && !(done && cnt == 0)) {
         const bool want_kv = !done && !kv_ready;
@@ -583,6 +584,7 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
         const bool hp = (bal >> 1) & 1u;
         const bool can_s = kv_ready && cnt - (hp ? 1 : 0) <= 1;
         if (!(hp || can_s)) {
+            if ((++idle & 15) != 0) continue;
             const bool give_up = *abort || clock64() - t_last > kWaitBudgetCycles;
             if (__any_sync(0xffffffffu, give_up)) {
                 if (lane == 0 && !*abort)
