@@ -56,13 +56,16 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by >8
 
 enum : int { kChunkNone = 0, kChunkBlock = 1, kChunkGather = 2 };
+// info flag: every row of the super tile takes every key of the chunk (a block
+// below the diagonal that all four query blocks take, outside A-shape)
+constexpr int kChunkWhole = 1 << 9;
 
 struct ChunkDesc {
-    int info;  // type | need << 4 | last << 8: what the MMA issuer reads, in one load
+    int info;  // type | need << 4 | last << 8 | whole << 9 (see kChunkWhole)
     int type, last, need, ncols;
     int b, m;  // block chunks: key block and its 4-bit query-block mask
-    int cols[kChunkKeys];
-    uint8_t cm[kChunkKeys];
+    int cols[kChunkKeys];      // gathers: the columns, ascending
+    uint64_t qmask[4];         // gathers: per query block, the columns it takes
 };
 
 struct GatherHeld {
@@ -195,6 +198,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// bits 0 .. k-1 set (none for k <= 0, all for k >= 64)
+__device__ __forceinline__ uint64_t low_bits(long long k) {
+    return k <= 0 ? 0ull : (k >= 64 ? ~0ull : (1ull << k) - 1ull);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -257,14 +265,14 @@ struct Producer {
         return wait(&bars.k_empty[s], par, nkv) && wait(&bars.v_empty[s], par, nkv);
     }
 
-    // one 64-key block with its query-block mask
-    __device__ void block(int b, int m) {
+    // one 64-key block with its query-block mask; `whole`: see kChunkWhole
+    __device__ void block(int b, int m, bool whole) {
         if (!ok) return;
         ChunkDesc* d = acquire_desc();
         if (!d) return;
         if (lane == 0) {
             const int need = ((m & 0x3) ? 1 : 0) | ((m & 0xC) ? 2 : 0);
-            d->info = kChunkBlock | (need << 4);
+            d->info = kChunkBlock | (need << 4) | (whole ? kChunkWhole : 0);
             d->type = kChunkBlock;
             d->last = 0;
             d->need = need;
@@ -296,25 +304,27 @@ struct Producer {
         if (!ok) return;
         ChunkDesc* d = acquire_desc();
         if (!d) return;
-        int need = 0;
-        for (int c = lane; c < kChunkKeys; c += 32) {
-            const bool v = c < n;
-            const int col = v ? held->cols[c] : held->cols[0];
-            const int cm = v ? held->cm[c] : 0;
-            d->cols[c] = col;
-            d->cm[c] = (uint8_t)cm;
-            need |= cm;
-        }
-        for (int off = 16; off >= 1; off >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, off);
+        // lane l holds columns l and l + 32; unused entries repeat a real column
+        const int cm0 = lane < n ? held->cm[lane] : 0;
+        const int cm1 = lane + 32 < n ? held->cm[lane + 32] : 0;
+        d->cols[lane] = lane < n ? held->cols[lane] : held->cols[0];
+        d->cols[lane + 32] = lane + 32 < n ? held->cols[lane + 32] : held->cols[0];
+        uint64_t qm[4];
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+            qm[qq] = (uint64_t)__ballot_sync(0xffffffffu, (cm0 >> qq) & 1) |
+                     ((uint64_t)__ballot_sync(0xffffffffu, (cm1 >> qq) & 1) << 32);
+        const int need = (qm[0] | qm[1] ? 1 : 0) | (qm[2] | qm[3] ? 2 : 0);
         if (lane == 0) {
-            const int nd = ((need & 0x3) ? 1 : 0) | ((need & 0xC) ? 2 : 0);
-            d->info = kChunkGather | (nd << 4);
+            d->info = kChunkGather | (need << 4);
             d->type = kChunkGather;
             d->last = 0;
-            d->need = nd;
+            d->need = need;
             d->ncols = n;
             d->b = -1;
             d->m = 0;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) d->qmask[qq] = qm[qq];
         }
         publish_desc();
         int st;
@@ -450,7 +460,8 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
             const int src = __ffs(bal) - 1;
             bal &= bal - 1;
             const int mm = __shfl_sync(0xffffffffu, m, src);
-            pr.block(base + src, mm);
+            pr.block(base + src, mm,
+                     mm == 0xF && base + src < qb0 && pattern != MI_PATTERN_ASHAPE);
         }
     }
 
@@ -682,6 +693,34 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
         const ChunkDesc& d = desc[di];
         const int type = d.type, last = d.last;
         if (type != kChunkNone && ((d.need >> x) & 1)) {
+            // The chunk's keys this row takes, one bit per column (known from the
+            // descriptor, so worked out while S is still being computed).  A
+            // warp's 32 rows lie in one 64-row query block, so a chunk that block
+            // does not take is dropped by the whole warp at once (P rows of zeros).
+            uint64_t keep = ~0ull;
+            unsigned kv = 1u;  // bit 0: some row of the warp takes the chunk; bit 1: some row drops a key
+            if (d.info & kChunkWhole) {
+            } else if (type == kChunkBlock) {
+                keep = 0;
+                if ((d.m >> qi) & 1) {
+                    const long long j0 = 64LL * d.b;
+                    keep = low_bits(i - j0 + 1);  // causal: columns <= i
+                    if (ashape)  // sink (j < sink) or local window (i - j < window)
+                        keep &= low_bits(p.sink - j0) | ~low_bits(i - j0 - p.window + 1);
+                }
+            } else {
+                // gathered columns ascend: those <= i form a prefix
+                int lo = 0, hi = d.ncols;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if ((long long)d.cols[mid] <= i) lo = mid + 1;
+                    else hi = mid;
+                }
+                keep = d.qmask[qi] & low_bits(lo);
+            }
+            if (!(d.info & kChunkWhole))
+                kv = __reduce_or_sync(0xffffffffu,
+                                      (keep != 0 ? 1u : 0u) | (keep != ~0ull ? 2u : 0u));
             const int b = n & 1;
             if (!__all_sync(0xffffffffu,
                             mbar_wait(&bars.s_full[2 * x + b], (n >> 1) & 1, abort))) {
@@ -691,96 +730,87 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
             }
             tc_fence_after();
             const uint32_t tS = __shfl_sync(0xffffffffu, tSlot + 64 * b, 0);
-            float v[kChunkKeys];
-            {
-                uint32_t r[32];
-                tmem_ld32(tS, r);
+            if (!(kv & 1u)) {
+                uint32_t z[32];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(r[u]);
-                tmem_ld32(tS + 32, r);
-#pragma unroll
-                for (int u = 0; u < 32; ++u) v[32 + u] = __uint_as_float(r[u]);
-            }
-            if (type == kChunkBlock) {
-                const int bit = (d.m >> qi) & 1;
-                const long long j0 = 64LL * d.b;
-                const bool full = bit && (j0 + 63 <= i) &&
-                                  (!ashape || j0 + 63 < p.sink || i - j0 < p.window);
-                if (!full) {
-#pragma unroll
-                    for (int c = 0; c < kChunkKeys; ++c) {
-                        const long long j = j0 + c;
-                        const bool keep =
-                            bit && j <= i && (!ashape || j < p.sink || i - j < p.window);
-                        if (!keep) v[c] = -INFINITY;
-                    }
-                }
+                for (int u = 0; u < 32; ++u) z[u] = 0u;
+                tmem_st32(tS, z);
             } else {
+                float v[kChunkKeys];
+                {
+                    uint32_t r[32];
+                    tmem_ld32(tS, r);
 #pragma unroll
-                for (int c = 0; c < kChunkKeys; ++c) {
-                    const bool keep = ((d.cm[c] >> qi) & 1) && (long long)d.cols[c] <= i;
-                    if (!keep) v[c] = -INFINITY;
+                    for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(r[u]);
+                    tmem_ld32(tS + 32, r);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) v[32 + u] = __uint_as_float(r[u]);
                 }
-            }
-            // raw scores: the scale (> 0) commutes with the max and is folded into
-            // the exponent below (one packed FFMA per pair)
-            float mq[2] = {fmaxf(v[0], v[1]), fmaxf(v[2], v[3])};
+                if (kv & 2u) {
 #pragma unroll
-            for (int c = 4; c < kChunkKeys; c += 4) {
-                mq[0] = fmax3(mq[0], v[c], v[c + 1]);
-                mq[1] = fmax3(mq[1], v[c + 2], v[c + 3]);
-            }
-            const float mx = fmaxf(mq[0], mq[1]) * cs;
-            // Lazy rescale: a row moves its reference max only when the max grew by
-            // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  O may be
-            // rescaled only once the slot's previous O += P V has run.  The TMEM
-            // accesses are .sync.aligned, so the whole warp takes the branch
-            // together; rows that do not need it scale by 1.
-            const bool want = mx > m + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, want)) {
-                const float alpha = want ? ex2(m - mx) : 1.f;  // 0 while m is -inf
-                if (n > 0) {
-                    const int pb = (n - 1) & 1;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + pb],
-                                                           ((n - 1) >> 1) & 1, abort))) {
-                        if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxO, g, 0);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint32_t o[32];
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        tmem_ld32(tO + 32 * c, o);
-#pragma unroll
-                        for (int u = 0; u < 32; ++u)
-                            o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-                        tmem_st32(tO + 32 * c, o);
-                    }
+                    for (int c = 0; c < kChunkKeys; ++c)
+                        if (!((keep >> c) & 1)) v[c] = -INFINITY;
                 }
-                l *= alpha;
-                if (want) m = mx;
-            }
-            const float mu = (m == -INFINITY) ? 0.f : m;
-            const uint64_t cs2 = f2_pack(cs, cs), nmu2 = f2_pack(-mu, -mu);
-            uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f),
-                                f2_pack(0.f, 0.f)};
-            uint32_t pk[32];
+                // raw scores: the scale (> 0) commutes with the max and is folded into
+                // the exponent below (one packed FFMA per pair)
+                float mq[2] = {fmaxf(v[0], v[1]), fmaxf(v[2], v[3])};
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const uint64_t x2 = f2_fma(f2_pack(v[2 * u], v[2 * u + 1]), cs2, nmu2);
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
-                const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
-                sum2[u & 3] = f2_add(sum2[u & 3], p2);
-                float p0, p1;
-                f2_unpack(p2, p0, p1);
-                pk[u] = pack_bf16(p0, p1);
+                for (int c = 4; c < kChunkKeys; c += 4) {
+                    mq[0] = fmax3(mq[0], v[c], v[c + 1]);
+                    mq[1] = fmax3(mq[1], v[c + 2], v[c + 3]);
+                }
+                const float mx = fmaxf(mq[0], mq[1]) * cs;
+                // Lazy rescale: a row moves its reference max only when the max grew by
+                // more than 2^8 (p <= 256 otherwise, exact after the final 1/l).  O may be
+                // rescaled only once the slot's previous O += P V has run.  The TMEM
+                // accesses are .sync.aligned, so the whole warp takes the branch
+                // together; rows that do not need it scale by 1.
+                const bool want = mx > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, want)) {
+                    const float alpha = want ? ex2(m - mx) : 1.f;  // 0 while m is -inf
+                    if (n > 0) {
+                        const int pb = (n - 1) & 1;
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + pb],
+                                                               ((n - 1) >> 1) & 1, abort))) {
+                            if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxO, g, 0);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        uint32_t o[32];
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            tmem_ld32(tO + 32 * c, o);
+#pragma unroll
+                            for (int u = 0; u < 32; ++u)
+                                o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+                            tmem_st32(tO + 32 * c, o);
+                        }
+                    }
+                    l *= alpha;
+                    if (want) m = mx;
+                }
+                const float mu = (m == -INFINITY) ? 0.f : m;
+                const uint64_t cs2 = f2_pack(cs, cs), nmu2 = f2_pack(-mu, -mu);
+                uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f),
+                                    f2_pack(0.f, 0.f)};
+                uint32_t pk[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const uint64_t x2 = f2_fma(f2_pack(v[2 * u], v[2 * u + 1]), cs2, nmu2);
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+                    sum2[u & 3] = f2_add(sum2[u & 3], p2);
+                    float p0, p1;
+                    f2_unpack(p2, p0, p1);
+                    pk[u] = pack_bf16(p0, p1);
+                }
+                tmem_st32(tS, pk);  // P over the first 32 columns of its S buffer
+                float s0, s1;
+                f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+                l += s0 + s1;
             }
-            tmem_st32(tS, pk);  // P over the first 32 columns of its S buffer
-            float s0, s1;
-            f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
-            l += s0 + s1;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars.p_full[2 * x + b]);
