@@ -8,8 +8,9 @@
 //   meanpool:  Qm[h][b] = mean of q rows 64b..64b+63 (fp64 sum, fp32 out),
 //              Km[g][b] likewise.  Pure HBM stream with 16-byte loads.
 //   bs_topk:   S[bq][bk] = scale * Qm[bq] . Km[bk] for bk <= bq (fp64 sum of
-//              exact fp32 products, ranked as fp32), kept on chip, then a
-//              block-wide radix top-k per query block, ascending output.
+//              exact fp32 products, ranked as fp32), register-tiled and kept
+//              on chip, then a warp-wide radix top-k per query block,
+//              ascending output.
 #include "internal.h"
 #include "topk.cuh"
 
@@ -52,28 +53,45 @@ __global__ void __launch_bounds__(kPoolThreads) meanpool_kernel(const bf16* __re
     }
 }
 
-constexpr int kMaxR = 16;
+constexpr int kMaxR = 16;       // query-block rows per CTA (fewer when the rows are long)
 constexpr int kTopkThreads = 256;
+constexpr int kKeyTile = 64;     // key blocks per shared-memory tile
+constexpr size_t kBsSmemCap = 227 * 1024;
 
 struct SmemKeys {
     const float* p;
     __device__ uint32_t operator()(int j) const { return float_order_key(p[j]); }
 };
 
+// Shared memory of one CTA: Qm rows [D][kMaxR] and a Km tile [D][kKeyTile],
+// both fp64; scores [R][stride] fp32; one 256-bin histogram per warp.
+template <int D>
+constexpr size_t bs_fixed_smem() {
+    return (size_t)D * kMaxR * 8 + (size_t)D * kKeyTile * 8 + (kTopkThreads / 32) * 256 * 4;
+}
+
+// CTA = R consecutive query blocks of one head.
+//  scores: warp w computes rows 2w and 2w+1, lane l key blocks 2l and 2l+1 of
+//          each 64-block tile, as fp64 sums of exact fp32 products over the
+//          d coordinates (operands widened once, on their way into shared
+//          memory); S = scale * sum, rounded to fp32 for ranking.
+//  top-k:  warp w selects rows w, w + 8, ... by a warp-wide radix select over
+//          its row of S, ties toward the lower block, output ascending.
 template <int D>
 __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     const float* __restrict__ qm, const float* __restrict__ km, int Hq, int Hkv, int nB,
     int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk,
     int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt) {
-    extern __shared__ __align__(16) float fsm[];
-    __shared__ TopkSmem ts;
+    extern __shared__ __align__(16) double dsm[];
+    double* Qs = dsm;                          // [D][kMaxR]
+    double* Ks = Qs + D * kMaxR;               // [D][kKeyTile]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + D * kKeyTile);  // [8][256]
+    float* S = reinterpret_cast<float*>(hist + (kTopkThreads / 32) * 256);  // [R][stride]
     const int pos = blockIdx.y;
     const int bq0 = blockIdx.x * R;
     const int nr = min(R, nB - bq0);
     const int ncand = bq0 + nr;
     const int stride = bq0 + R;
-    float* Qs = fsm;           // [R][D]
-    float* S = fsm + R * D;    // [R][stride]
     const int qh = head_qh(heads.e[pos]);
     const int g = kv_head_of(qh, Hq, Hkv);
     // Km is stored per KV head in use; kvpos maps KV head -> its row in Km
@@ -81,57 +99,74 @@ __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     for (int t = 0; t < kvmap_n; ++t)
         if (head_qh(kvpos.e[t]) == g) gi = t;
     const float* kmg = km + (size_t)gi * nB * D;
-
-    for (int t = threadIdx.x; t < nr * D; t += blockDim.x)
-        Qs[t] = qm[((size_t)pos * nB + bq0) * D + t];
-    __syncthreads();
-
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int bk = warp; bk < ncand; bk += kTopkThreads / 32) {
-        double acc[kMaxR];
-#pragma unroll
-        for (int r = 0; r < kMaxR; ++r) acc[r] = 0.0;
-#pragma unroll
-        for (int u = 0; u < D / 32; ++u) {
-            const int t = lane + 32 * u;
-            const double kv = (double)kmg[(size_t)bk * D + t];
-#pragma unroll
-            for (int r = 0; r < kMaxR; ++r)
-                if (r < nr) acc[r] = fma((double)Qs[r * D + t], kv, acc[r]);
+
+    // consecutive threads fill consecutive shared words (no bank conflicts)
+    for (int t = threadIdx.x; t < kMaxR * D; t += blockDim.x) {
+        const int r = t % kMaxR, c = t / kMaxR;
+        Qs[c * kMaxR + r] = r < nr ? (double)qm[((size_t)pos * nB + bq0 + r) * D + c] : 0.0;
+    }
+    for (int kt0 = 0; kt0 < ncand; kt0 += kKeyTile) {
+        __syncthreads();  // the previous tile has been used
+        for (int t = threadIdx.x; t < kKeyTile * (D / 4); t += blockDim.x) {
+            const int kb = t % kKeyTile, c4 = t / kKeyTile;
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kt0 + kb < ncand)
+                f = *reinterpret_cast<const float4*>(kmg + (size_t)(kt0 + kb) * D + 4 * c4);
+            Ks[(4 * c4 + 0) * kKeyTile + kb] = f.x;
+            Ks[(4 * c4 + 1) * kKeyTile + kb] = f.y;
+            Ks[(4 * c4 + 2) * kKeyTile + kb] = f.z;
+            Ks[(4 * c4 + 3) * kKeyTile + kb] = f.w;
         }
-#pragma unroll
-        for (int r = 0; r < kMaxR; ++r) {
-            if (r >= nr) break;
-            double a = acc[r];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-            if (lane == 0) S[r * stride + bk] = (float)(a * scale);
+        __syncthreads();
+        if (2 * warp < nr) {
+            double a00 = 0.0, a01 = 0.0, a10 = 0.0, a11 = 0.0;
+#pragma unroll 8
+            for (int c = 0; c < D; ++c) {
+                const double2 qv = *reinterpret_cast<const double2*>(Qs + c * kMaxR + 2 * warp);
+                const double2 kv = *reinterpret_cast<const double2*>(Ks + c * kKeyTile + 2 * lane);
+                a00 = fma(qv.x, kv.x, a00);
+                a01 = fma(qv.x, kv.y, a01);
+                a10 = fma(qv.y, kv.x, a10);
+                a11 = fma(qv.y, kv.y, a11);
+            }
+            const int k0 = kt0 + 2 * lane, r0 = 2 * warp;
+            if (k0 < ncand) {
+                S[r0 * stride + k0] = (float)(a00 * scale);
+                if (r0 + 1 < nr) S[(r0 + 1) * stride + k0] = (float)(a10 * scale);
+            }
+            if (k0 + 1 < ncand) {
+                S[r0 * stride + k0 + 1] = (float)(a01 * scale);
+                if (r0 + 1 < nr) S[(r0 + 1) * stride + k0 + 1] = (float)(a11 * scale);
+            }
         }
     }
     __syncthreads();
 
-    for (int r = 0; r < nr; ++r) {
+    for (int r = warp; r < nr; r += kTopkThreads / 32) {
         const int bq = bq0 + r;
         const int n = bq + 1;
         const int kk = min(topk, n);
         int32_t* o = blk_idx + ((size_t)pos * nB + bq) * topk;
-        for (int t = kk + threadIdx.x; t < topk; t += blockDim.x) o[t] = -1;
-        if (threadIdx.x == 0) blk_cnt[(size_t)pos * nB + bq] = kk;
+        for (int t = kk + lane; t < topk; t += 32) o[t] = -1;
+        if (lane == 0) blk_cnt[(size_t)pos * nB + bq] = kk;
         if (kk == n) {
-            for (int t = threadIdx.x; t < n; t += blockDim.x) o[t] = t;
+            for (int t = lane; t < n; t += 32) o[t] = t;
         } else if (kk > 0) {
             SmemKeys get{S + r * stride};
             uint32_t thr;
             int need_eq;
-            block_radix_select(get, n, kk, ts, thr, need_eq);
-            block_select_compact(get, n, kk, thr, need_eq, ts, o);
+            warp_radix_select(get, n, kk, hist + warp * 256, thr, need_eq);
+            warp_select_compact(get, n, kk, thr, need_eq, o);
         }
-        __syncthreads();
     }
 }
 
+// Rows per CTA: as many (up to kMaxR) as the score rows leave room for.
+template <int D>
 int rows_per_cta(int nB) {
-    int R = 24576 / (nB > 0 ? nB : 1);
+    const size_t room = kBsSmemCap - bs_fixed_smem<D>() - 1024;
+    int R = (int)(room / (4 * (size_t)(nB + kMaxR)));
     if (R > kMaxR) R = kMaxR;
     if (R < 1) R = 1;
     return R;
@@ -150,8 +185,8 @@ cudaError_t launch_bs_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, do
         if (used[g]) kvs.e[kvs.n++] = pack_head(g, 0, 0);
     meanpool_kernel<D><<<dim3(nB, heads.n), kPoolThreads, 0, st>>>(q, N, nB, heads, ws.qm);
     meanpool_kernel<D><<<dim3(nB, kvs.n), kPoolThreads, 0, st>>>(k, N, nB, kvs, ws.km);
-    const int R = rows_per_cta(nB);
-    const size_t smem = ((size_t)R * D + (size_t)R * (nB + R)) * sizeof(float);
+    const int R = rows_per_cta<D>(nB);
+    const size_t smem = bs_fixed_smem<D>() + (size_t)R * (nB + R) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bs_topk_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -115,4 +115,78 @@ __device__ void block_select_compact(const Get& get, int n, int k, uint32_t thr,
     }
 }
 
+// ---- one warp per selection (many short rows at once), same contract as above.
+// `hist` is this warp's own 256-entry shared histogram.
+template <class Get>
+__device__ void warp_radix_select(const Get& get, int n, int k, uint32_t* hist, uint32_t& thr,
+                                  int& need_eq) {
+    const int lane = threadIdx.x & 31;
+    uint32_t prefix = 0, mask = 0;
+    int rem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        __syncwarp();
+        for (int j = lane; j < n; j += 32) {
+            const uint32_t key = get(j);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        // lane l owns bins 255-8l down to 248-8l; a scan over the lanes gives the
+        // count above each lane's bins, so one lane holds the bin where the
+        // running count from the top reaches `rem`
+        int c[8], sum = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            c[u] = (int)hist[255 - 8 * lane - u];
+            sum += c[u];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const int above = incl - sum;
+        const unsigned who = __ballot_sync(0xffffffffu, above < rem && rem <= incl);
+        const int src = who ? __ffs(who) - 1 : 31;
+        int bsel = 0, left = rem - above;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (left <= c[u]) {
+                bsel = 255 - 8 * lane - u;
+                break;
+            }
+            left -= c[u];
+        }
+        bsel = __shfl_sync(0xffffffffu, bsel, src);
+        rem = __shfl_sync(0xffffffffu, left, src);
+        prefix |= (uint32_t)bsel << shift;
+        mask |= 255u << shift;
+        __syncwarp();
+    }
+    thr = prefix;
+    need_eq = rem;
+}
+
+template <class Get>
+__device__ void warp_select_compact(const Get& get, int n, int k, uint32_t thr, int need_eq,
+                                    int32_t* out) {
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    int eq_base = 0, sel_base = 0;
+    for (int base = 0; base < n && sel_base < k; base += 32) {
+        const int j = base + lane;
+        const uint32_t key = j < n ? get(j) : 0u;
+        const bool gt = j < n && key > thr;
+        const bool eq = j < n && key == thr;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const bool sel = gt || (eq && eq_base + __popc(eqm & below) < need_eq);
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        const int pos = sel_base + __popc(selm & below);
+        if (sel && pos < k) out[pos] = j;
+        eq_base += __popc(eqm);
+        sel_base += __popc(selm);
+    }
+}
+
 }  // namespace minfer
