@@ -28,6 +28,7 @@
 #include <cstring>
 #include <cudaTypedefs.h>
 
+#include "exp2_poly.h"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -195,6 +196,27 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair on the FMA pipe (steps and constants in exp2_poly.h).  A
+// quarter of the softmax exponentials take this path: the two slots' softmax
+// warps share the MUFU unit, which is otherwise the busiest pipe of the loop.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    float a, b;
+    f2_unpack(x2, a, b);
+    const uint64_t xc = f2_pack(fmaxf(a, kExp2Clamp), fmaxf(b, kExp2Clamp));
+    const uint64_t t = f2_add(xc, f2_pack(kExp2Round, kExp2Round));
+    const uint64_t tn = f2_add(t, f2_pack(-kExp2Round, -kExp2Round));
+    const uint64_t fr = f2_fma(tn, f2_pack(-1.f, -1.f), xc);
+    uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), fr, f2_pack(kExp2C2, kExp2C2));
+    q = f2_fma(q, fr, f2_pack(kExp2C1, kExp2C1));
+    q = f2_fma(q, fr, f2_pack(kExp2C0, kExp2C0));
+    uint32_t qlo, qhi, tlo, thi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(qlo), "=r"(qhi) : "l"(q));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(tlo), "=r"(thi) : "l"(t));
+    uint64_t r;  // 2^n by adding n (low bits of t) to the exponent field
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(qlo + (tlo << 23)), "r"(qhi + (thi << 23)));
     return r;
 }
 
@@ -800,7 +822,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                     const uint64_t x2 = f2_fma(f2_pack(v[2 * u], v[2 * u + 1]), cs2, nmu2);
                     float x0, x1;
                     f2_unpack(x2, x0, x1);
-                    const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+                    const uint64_t p2 = (u % 4 == 3) ? exp2_poly2(x2) : f2_pack(ex2(x0), ex2(x1));
                     sum2[u & 3] = f2_add(sum2[u & 3], p2);
                     float p0, p1;
                     f2_unpack(p2, p0, p1);
