@@ -43,6 +43,16 @@ __device__ void load_rows_T(double* dst, const bf16* base, long long row0, int n
     }
 }
 
+// Thread -> 4x4 sub-tile of the 64x64 (rows x keys) tile: warp w covers row
+// groups 8*(w/4) .. +7 and key groups 4*(w%4) .. +3, lane l row group
+// l/4 and key group l%4 within them.  Per step a warp then reads 8 distinct
+// 32-byte Q pieces and 4 distinct K pieces (4 conflict-free wavefronts).
+__device__ __forceinline__ void tile_coords(int& ty, int& tx) {
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    ty = (w >> 2) * 8 + (l >> 2);
+    tx = (w & 3) * 4 + (l & 3);
+}
+
 // acc[a][b] = sum_t Qs[t][4ty+a] * Ks[t][4tx+b]
 template <int D>
 __device__ __forceinline__ void dot_4x4(const double* Qs, const double* Ks, int ty, int tx,
@@ -93,7 +103,8 @@ __global__ void __launch_bounds__(kThreads) vs_rowstat_kernel(const bf16* __rest
     const int g = kv_head_of(qh, Hq, Hkv);
     const int r0 = rt * 64, nr = min(64, L - r0);
     const long long i0 = (long long)N - L + r0;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    int tx, ty;
+    tile_coords(ty, tx);
 
     load_rows_T<D>(Qs, q + (long long)qh * N * D, i0, nr);
     const int jb = c * kVsChunk, je = min(N, jb + kVsChunk);
@@ -129,20 +140,31 @@ __global__ void __launch_bounds__(kThreads) vs_rowstat_kernel(const bf16* __rest
             }
         }
     }
+    // merge the 16 key groups of each row: 4 lanes of a warp, then 4 warps
+    __syncthreads();  // Ks is reused as the merge buffer [4][64] x (m, l)
+    double* red = Ks;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) {
+        for (int off = 2; off >= 1; off >>= 1) {
             const double m2 = __shfl_xor_sync(0xffffffffu, m[a], off);
             const double l2 = __shfl_xor_sync(0xffffffffu, l[a], off);
             merge_ml(m[a], l[a], m2, l2);
         }
-        const int rr = ty * 4 + a;
-        if (tx == 0 && rr < nr) {
-            const size_t o = ((size_t)pos * L + r0 + rr) * nchunks + c;
-            m_part[o] = m[a];
-            l_part[o] = l[a];
+        if ((threadIdx.x & 3) == 0) {
+            const int rr = ty * 4 + a, wq = (threadIdx.x >> 5) & 3;
+            red[(wq * 64 + rr) * 2] = m[a];
+            red[(wq * 64 + rr) * 2 + 1] = l[a];
         }
+    }
+    __syncthreads();
+    if (threadIdx.x < nr) {
+        const int rr = threadIdx.x;
+        double mm = red[rr * 2], ll = red[rr * 2 + 1];
+        for (int wq = 1; wq < 4; ++wq) merge_ml(mm, ll, red[(wq * 64 + rr) * 2], red[(wq * 64 + rr) * 2 + 1]);
+        const size_t o = ((size_t)pos * L + r0 + rr) * nchunks + c;
+        m_part[o] = mm;
+        l_part[o] = ll;
     }
 }
 
@@ -169,7 +191,8 @@ __global__ void __launch_bounds__(kThreads) vs_colslash_kernel(
     const long long o_hi = (c == 0) ? (long long)N - 1 : (long long)N - L - jb;
     const long long o_lo = max(0LL, (long long)N - L - je + 1);
     const int n_own = o_hi >= o_lo ? (int)(o_hi - o_lo + 1) : 0;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    int tx, ty;
+    tile_coords(ty, tx);
 
     for (int r = threadIdx.x; r < L; r += blockDim.x) {
         double mm = -DBL_MAX, ll = 0.0;
