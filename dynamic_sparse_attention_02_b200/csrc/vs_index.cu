@@ -53,6 +53,35 @@ __device__ __forceinline__ void tile_coords(int& ty, int& tx) {
     tx = (w & 3) * 4 + (l & 3);
 }
 
+// The same 64-row tile in two steps, so that the global loads of the next
+// tile can be in flight while the current one is used: fetch into registers
+// (kTileChunks 16-byte pieces per thread), then widen and store.
+template <int D>
+struct TileRegs {
+    static constexpr int kChunks = D / 8;
+    static constexpr int kPer = 64 * kChunks / kThreads;
+    uint4 v[kPer];
+    __device__ void fetch(const bf16* base, long long row0, int nvalid) {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int idx = threadIdx.x + u * kThreads;
+            const int r = idx & 63, c = idx >> 6;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (r < nvalid) v[u] = *reinterpret_cast<const uint4*>(base + (row0 + r) * D + c * 8);
+        }
+    }
+    __device__ void store_T(double* dst) const {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int idx = threadIdx.x + u * kThreads;
+            const int r = idx & 63, c = idx >> 6;
+            const bf16* e = reinterpret_cast<const bf16*>(&v[u]);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) dst[(c * 8 + w) * 64 + r] = (double)__bfloat162float(e[w]);
+        }
+    }
+};
+
 // acc[a][b] = sum_t Qs[t][4ty+a] * Ks[t][4tx+b]
 template <int D>
 __device__ __forceinline__ void dot_4x4(const double* Qs, const double* Ks, int ty, int tx,
@@ -114,11 +143,15 @@ __global__ void __launch_bounds__(kThreads) vs_rowstat_kernel(const bf16* __rest
         m[a] = -DBL_MAX;
         l[a] = 0.0;
     }
+    const bf16* kb = k + (long long)g * N * D;
+    TileRegs<D> next;
+    next.fetch(kb, jb, min(64, je - jb));
     for (int j0 = jb; j0 < je; j0 += 64) {
         if (j0 > i0 + nr - 1) break;  // every key past every row: causal
         __syncthreads();
-        load_rows_T<D>(Ks, k + (long long)g * N * D, j0, min(64, je - j0));
+        next.store_T(Ks);
         __syncthreads();
+        if (j0 + 64 < je && j0 + 64 <= i0 + nr - 1) next.fetch(kb, j0 + 64, min(64, je - j0 - 64));
         double acc[4][4];
         dot_4x4<D>(Qs, Ks, ty, tx, acc);
 #pragma unroll
@@ -209,11 +242,15 @@ __global__ void __launch_bounds__(kThreads) vs_colslash_kernel(
         const long long i0 = (long long)N - L + r0;
         __syncthreads();
         load_rows_T<D>(Qs, q + (long long)qh * N * D, i0, nr);
+        const bf16* kb = k + (long long)g * N * D;
+        TileRegs<D> next;
+        next.fetch(kb, jb, min(64, jh - jb));
         for (int j0 = jb; j0 < jh; j0 += 64) {
             if (j0 > i0 + nr - 1) break;
             __syncthreads();
-            load_rows_T<D>(Ks, k + (long long)g * N * D, j0, min(64, jh - j0));
+            next.store_T(Ks);
             __syncthreads();
+            if (j0 + 64 < jh && j0 + 64 <= i0 + nr - 1) next.fetch(kb, j0 + 64, min(64, jh - j0 - 64));
             double acc[4][4];
             dot_4x4<D>(Qs, Ks, ty, tx, acc);
 #pragma unroll
