@@ -173,6 +173,19 @@ def vs_useful_flops(v_idx, s_idx, N, d):
     return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
 
 
+def ashape_tiles(N, sink, window):
+    """64x64 causal tiles an A-shape head computes: key block b of query block qb
+    holds a sink key (64 b < sink) or a key inside the local window of some row
+    (64 (qb - b) - 63 < window)."""
+    nB = N // 64
+    qb = np.arange(nB)
+    a = np.minimum(qb + 1, -(-sink // 64))        # sink blocks: b < ceil(sink / 64)
+    dmax = -(-(window + 63) // 64) - 1            # window blocks: qb - b <= dmax
+    lo = np.maximum(0, qb - dmax)
+    both = np.maximum(0, np.minimum(a, qb + 1) - lo)
+    return int(np.sum(a + (qb - lo + 1) - both))
+
+
 # ----------------------------------------------------------------- oracle timing
 
 def oracle_sample(w, x, budget_s, rng, h=0, min_rows=32, max_rows=16384):
@@ -369,14 +382,28 @@ def run_minfer(args):
     useful = 0.0
     tiles = 0
     cols = 0
-    if n_vs == w.Hq:
-        v_idx, s_idx = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size)
+    pat = np.asarray(pattern)
+    vs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_VS]
+    bs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_BS]
+    n_ash = int(np.sum(pat == synth.PATTERN_ASHAPE))
+    if vs_heads:
+        v_idx, s_idx = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size,
+                                     heads=vs_heads)
         vi, si = v_idx.cpu().numpy(), s_idx.cpu().numpy()
-        for h in range(w.Hq):
-            f, t, c = vs_useful_flops(vi[h], si[h], w.N, w.d)
+        for i in range(len(vs_heads)):
+            f, t, c = vs_useful_flops(vi[i], si[i], w.N, w.d)
             useful += f
             tiles += t
             cols += c
+    if bs_heads:
+        _, blk_cnt = B.mi_bs_index(q, k, w.topk_blocks, heads=bs_heads)
+        t = int(blk_cnt.sum().item())
+        useful += 4.0 * w.d * 64 * 64 * t
+        tiles += t
+    if n_ash:
+        t = ashape_tiles(w.N, w.sink, w.window) * n_ash
+        useful += 4.0 * w.d * 64 * 64 * t
+        tiles += t
     dense_eq = 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))

@@ -25,3 +25,18 @@ def test_vs_useful_flops_matches_brute_force():
             v = rng.integers(-1, N, size=rng.integers(0, 40)).astype(np.int32)
             s = rng.integers(-1, N, size=rng.integers(0, 30)).astype(np.int32)
             assert bench.vs_useful_flops(v, s, N, 128) == brute(v, s, N, 128)
+
+
+def test_ashape_tile_count_matches_brute_force():
+    """The closed-form count of 64x64 tiles an A-shape head computes (bench FLOP
+    accounting) equals a direct count over every causal (query block, key block)."""
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        N = 64 * int(rng.integers(1, 70))
+        sink = int(rng.integers(0, 300))
+        window = int(rng.integers(0, 1500))
+        nB = N // 64
+        qb = np.arange(nB)[:, None]
+        b = np.arange(nB)[None, :]
+        want = int(np.sum((b <= qb) & ((64 * b < sink) | (64 * (qb - b) - 63 < window))))
+        assert bench.ashape_tiles(N, sink, window) == want
