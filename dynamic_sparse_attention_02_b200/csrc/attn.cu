@@ -11,7 +11,11 @@
 // blocks), held as two 128-row slots.  The producer enumerates the item's
 // key chunks -- one 64-key block, or up to 64 gathered vertical columns --
 // each with a 4-bit mask (one bit per query block); a chunk is computed for
-// the slots whose bits it carries, and rows whose bit is clear see -inf.
+// the slots whose bits it carries.  Each softmax row turns the descriptor
+// into a 64-bit mask of the keys it takes (causal limit, A-shape sink and
+// window, gathered columns); a warp whose query block does not take the
+// chunk writes zero P rows and skips the exponentials, and chunks that every
+// row takes whole are flagged so that they skip the mask step.
 //   warps 0-3  softmax, slot 0 (TMEM lanes 0-127 = rows 0-127)
 //   warps 4-7  softmax, slot 1 (rows 128-255)
 //   warp 8     producer: chunk list + TMA loads (cp.async gathers), 4 deep
@@ -19,7 +23,8 @@
 // Each slot double-buffers S in TMEM, so the tensor core computes S(n+1)
 // while the softmax works on S(n); O += P(n) V(n) follows once P(n) is
 // ready.  A slot's softmax therefore runs back to back, whether or not the
-// other slot needs the same chunk.
+// other slot needs the same chunk.  The exponentials run on MUFU, a quarter
+// of them on the FMA pipe (exp2_poly.h).
 //
 // TMEM (512 columns): slot x owns [256x, 256x+256): S buffers 0 and 1 at
 // +0 and +64 (64 columns each; P, bf16 pairs, reuses the first 32), O at
