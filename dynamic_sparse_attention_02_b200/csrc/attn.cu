@@ -273,9 +273,31 @@ struct Producer {
         }
         return w;
     }
+    // A wait costs about 200 cycles even on a long-completed phase, and the
+    // next chunk needs three (its descriptor slot, K stage and V stage free).
+    // One non-blocking probe across lanes 0-2 checks all three; when they have
+    // completed, acquire_desc and acquire_kv skip their waits for this chunk.
+    bool free_known = false;
+    __device__ void probe_next() {
+        uint64_t* b = bars.q_full;
+        uint32_t par = 0;
+        bool live = false;
+        if (lane == 0 && pub >= kDescRing) {
+            b = &bars.desc_empty[pub % kDescRing];
+            par = ((pub / kDescRing) - 1) & 1;
+            live = true;
+        } else if ((lane == 1 || lane == 2) && nkv >= kStages) {
+            b = lane == 1 ? &bars.k_empty[nkv % kStages] : &bars.v_empty[nkv % kStages];
+            par = ((nkv / kStages) - 1) & 1;
+            live = true;
+        }
+        const bool hit = mbar_test_wait(b, par) || !live;
+        free_known = __all_sync(0xffffffffu, hit);
+    }
     __device__ ChunkDesc* acquire_desc() {
         const int i = pub % kDescRing;
-        if (pub >= kDescRing && !wait(&bars.desc_empty[i], ((pub / kDescRing) - 1) & 1, pub))
+        if (pub >= kDescRing && !free_known &&
+            !wait(&bars.desc_empty[i], ((pub / kDescRing) - 1) & 1, pub))
             return nullptr;
         return &desc[i];
     }
@@ -287,7 +309,9 @@ struct Producer {
     // the stage of the next descriptor, once its previous K and V are released
     __device__ bool acquire_kv(int& s) {
         s = nkv % kStages;
-        if (nkv < kStages) return true;
+        const bool known = free_known;  // good for this chunk only
+        free_known = false;
+        if (nkv < kStages || known) return true;
         const int par = ((nkv / kStages) - 1) & 1;
         return wait(&bars.k_empty[s], par, nkv) && wait(&bars.v_empty[s], par, nkv);
     }
@@ -295,6 +319,7 @@ struct Producer {
     // one 64-key block with its query-block mask; `whole`: see kChunkWhole
     __device__ void block(int b, int m, bool whole) {
         if (!ok) return;
+        probe_next();
         ChunkDesc* d = acquire_desc();
         if (!d) return;
         if (lane == 0) {
@@ -329,6 +354,7 @@ struct Producer {
     // up to 64 gathered columns
     __device__ void gather(int n) {
         if (!ok) return;
+        probe_next();
         ChunkDesc* d = acquire_desc();
         if (!d) return;
         // lane l holds columns l and l + 32; unused entries repeat a real column
