@@ -165,6 +165,25 @@ def test_vs_attn_unsorted_duplicates_and_empty_rows():
     assert torch.all(out[1, :5] == 0) and torch.all(torch.isneginf(lse[1, :5]))
 
 
+def test_vs_attn_gathered_columns_inside_query_blocks():
+    """Many vertical columns, most of them inside the rows' own query blocks,
+    with only far slash diagonals (so no diagonal tile covers them): each
+    gathered chunk holds columns of several query blocks, and every row must
+    take exactly the gathered columns j <= i.  Rows before the first column
+    and every diagonal are empty."""
+    q, k, v = rand_bf16(2, 1, 1088, 128, 21)
+    rng = np.random.default_rng(5)
+    vi = np.stack([rng.choice(1088, 400, replace=False) for _ in range(2)]).astype(np.int32)
+    si = np.array([[700, 901], [512, 640]], np.int32)
+    out, lse = B.mi_vs_sparse_attn(q, k, v, torch.from_numpy(vi).cuda(),
+                                   torch.from_numpy(si).cuda())
+    torch.cuda.synchronize()
+    for h in range(2):
+        qs, ks_, vs_ = head_slices(q, k, v, h)
+        ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, np.unique(vi[h]), np.unique(si[h]))
+        check_attn(out[h], lse[h], ro, rl, what=f"vs gathered h{h}")
+
+
 def test_vs_attn_counts_out_of_range_entries():
     q, k, v = rand_bf16(1, 1, 256, 64, 14)
     vi = torch.tensor([[3, 256, -7, 9]], dtype=torch.int32, device="cuda")
