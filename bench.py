@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 ATTN_SOURCES = ["attn.cu", "ptx.cuh", "internal.h"]
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -64,7 +64,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0,
                     help="approximate CPU seconds for the oracle baseline sample")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------- helpers
@@ -269,31 +269,56 @@ def config_of(w):
                    " > 126 MB); no flush")}
 
 
+class Ranks:
+    """One process per GPU, launched by torchrun: rank and world size from its
+    environment, and a process group for the barriers around the timed region
+    and the max-over-ranks step time (NCCL on the GPU machine; the tests drive the
+    same code over gloo on CPU).  The layer is run as independent replicas:
+    no collective touches the data path."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=300):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self.dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max_over_ranks(self, val):
+        if self.dist is None:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def job_value(ms_step_max, world):
+    """Whole-job ms per layer: `world` replicas each finish one layer per step,
+    timed by the slowest rank."""
+    return ms_step_max / world
+
+
 def run_minfer(args):
     from dynamic_sparse_attention_02_b200 import binding as B
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
-        torch.cuda.set_device(0)
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     dev = torch.device("cuda", torch.cuda.current_device())
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(val):
-        if dist is None:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
     w = workload_of(args)
     log(f"generating {w.name} (N={w.N})")
@@ -399,7 +424,7 @@ def run_minfer(args):
         barrier()
         ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e)
         log(f"e2e {ms_e2e:.2f} ms/step")
-        e2e = {"value": ms_e2e / world, "unit": UNIT,
+        e2e = {"value": job_value(ms_e2e, world), "unit": UNIT,
                "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                "d2h_bytes_per_step": int(hout.numel() * 2), "steps": n_e2e}
         assert torch.equal(hout, out.cpu()), "e2e output differs from the device output"
@@ -447,7 +472,7 @@ def run_minfer(args):
             cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                    "sample": desc}
         line = {
-            "metric": METRIC, "value": ms_step_max / world, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": job_value(ms_step_max, world), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step_max,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config_of(w),
@@ -468,9 +493,7 @@ def run_minfer(args):
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
