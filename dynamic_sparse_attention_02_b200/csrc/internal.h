@@ -53,6 +53,8 @@ constexpr int kVsChunk = 1024;  // keys per CTA in the score passes
 struct VsIndexWs {
     double* m_part;  // [n_heads][L][nchunks]
     double* l_part;
+    double* mrow;    // [n_heads][L] merged row max
+    double* linv;    // [n_heads][L] 1 / merged row sum
     float* vscore;   // [n_heads][N]
     float* sscore;   // [n_heads][N]
 };

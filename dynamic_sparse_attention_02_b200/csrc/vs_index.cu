@@ -12,7 +12,9 @@
 // products of bf16 inputs are exact in fp64, so the scores agree with an
 // fp64 evaluation to rounding level and the ranking matches it):
 //   pass 1 (vs_rowstat): per key chunk, per row, the partial max and sum;
-//   pass 2 (vs_colslash): combine the partials, recompute the probabilities
+//   merge (vs_rowmerge): once per head, the partials into each row's final
+//     max and 1/sum;
+//   pass 2 (vs_colslash): recompute the probabilities
 //     and reduce them into column sums and diagonal sums in a fixed order
 //     (deterministic).  A chunk owns the diagonals whose first key falls in
 //     it and recomputes the L-1 keys past its end to finish them.
@@ -201,11 +203,26 @@ __global__ void __launch_bounds__(kThreads) vs_rowstat_kernel(const bf16* __rest
     }
 }
 
+// Final per-row normaliser of every listed head, merged once from the chunk
+// partials: mrow = max, linv = 1 / sum (0 for a row with no key).
+__global__ void vs_rowmerge_kernel(const double* __restrict__ m_part,
+                                                        const double* __restrict__ l_part, int L,
+                                                        int nchunks, double* mrow, double* linv) {
+    const int pos = blockIdx.x;
+    for (int r = threadIdx.x; r < L; r += blockDim.x) {
+        double mm = -DBL_MAX, ll = 0.0;
+        const size_t base = ((size_t)pos * L + r) * nchunks;
+        for (int cc = 0; cc < nchunks; ++cc) merge_ml(mm, ll, m_part[base + cc], l_part[base + cc]);
+        mrow[(size_t)pos * L + r] = mm;
+        linv[(size_t)pos * L + r] = ll > 0.0 ? 1.0 / ll : 0.0;
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads) vs_colslash_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k, int Hq, int Hkv, int N, int L,
-    int nchunks, HeadList heads, double scale, const double* __restrict__ m_part,
-    const double* __restrict__ l_part, float* vscore, float* sscore) {
+    int nchunks, HeadList heads, double scale, const double* __restrict__ mrow_g,
+    const double* __restrict__ linv_g, float* vscore, float* sscore) {
     extern __shared__ __align__(16) double sm[];
     double* Qs = sm;
     double* Ks = Qs + D * 64;
@@ -228,11 +245,8 @@ __global__ void __launch_bounds__(kThreads) vs_colslash_kernel(
     tile_coords(ty, tx);
 
     for (int r = threadIdx.x; r < L; r += blockDim.x) {
-        double mm = -DBL_MAX, ll = 0.0;
-        const size_t base = ((size_t)pos * L + r) * nchunks;
-        for (int cc = 0; cc < nchunks; ++cc) merge_ml(mm, ll, m_part[base + cc], l_part[base + cc]);
-        mrow[r] = mm;
-        linv[r] = ll > 0.0 ? 1.0 / ll : 0.0;
+        mrow[r] = mrow_g[(size_t)pos * L + r];
+        linv[r] = linv_g[(size_t)pos * L + r];
     }
     for (int t = threadIdx.x; t < kVsChunk; t += blockDim.x) vacc[t] = 0.0;
     for (int t = threadIdx.x; t < n_own; t += blockDim.x) sacc[t] = 0.0;
@@ -350,8 +364,9 @@ cudaError_t launch_vs_index_d(const bf16* q, const bf16* k, int Hq, int Hkv, int
         return e;
     vs_rowstat_kernel<D><<<dim3(nchunks, n, nrt), kThreads, sm1, st>>>(
         q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.m_part, ws.l_part);
+    vs_rowmerge_kernel<<<n, 64, 0, st>>>(ws.m_part, ws.l_part, L, nchunks, ws.mrow, ws.linv);
     vs_colslash_kernel<D><<<dim3(nchunks, n), kThreads, sm2, st>>>(
-        q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.m_part, ws.l_part, vsc, ssc);
+        q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.mrow, ws.linv, vsc, ssc);
     topk_rows_kernel<<<n, 1024, 0, st>>>(vsc, N, kv, v_idx, kv);
     topk_rows_kernel<<<n, 1024, 0, st>>>(ssc, N, ks, s_idx, ks);
     return cudaGetLastError();
@@ -365,6 +380,8 @@ VsIndexWs carve_vs_index(WsCarver& c, int n_heads, int N, int L, bool need_vscor
     VsIndexWs w{};
     w.m_part = c.take<double>((size_t)n_heads * L * nchunks);
     w.l_part = c.take<double>((size_t)n_heads * L * nchunks);
+    w.mrow = c.take<double>((size_t)n_heads * L);
+    w.linv = c.take<double>((size_t)n_heads * L);
     w.vscore = need_vscore ? c.take<float>((size_t)n_heads * N) : nullptr;
     w.sscore = need_sscore ? c.take<float>((size_t)n_heads * N) : nullptr;
     return w;
