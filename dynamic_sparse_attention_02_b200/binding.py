@@ -20,8 +20,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libminfer.so")
 
 MI_OK, MI_ERR_INVALID_ARG, MI_ERR_UNSUPPORTED, MI_ERR_WORKSPACE, MI_ERR_CUDA = range(5)
-MI_PATTERN_ASHAPE, MI_PATTERN_VS, MI_PATTERN_BS = 0, 1, 2
+MI_PATTERN_ASHAPE, MI_PATTERN_VS, MI_PATTERN_BS, MI_PATTERN_DENSE = 0, 1, 2, 3
 MI_OP_VS_INDEX, MI_OP_BS_INDEX, MI_OP_VS_ATTN, MI_OP_BS_ATTN, MI_OP_ASHAPE_ATTN = 1, 2, 3, 4, 5
+MI_OP_DENSE_ATTN = 6
 MI_STAGE_START, MI_STAGE_INDEX_DONE, MI_STAGE_PREP_DONE, MI_STAGE_ATTN_DONE, MI_STAGE_EVENTS = (
     0, 1, 2, 3, 4)
 MI_MAX_HEADS = 256
@@ -31,7 +32,7 @@ MI_BLOCK = 64
 EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
            "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
-           "mi_vs_index_static"]
+           "mi_vs_index_static", "mi_dense_attn"]
 
 
 class MinferError(RuntimeError):
@@ -79,6 +80,7 @@ def _lib_handle():
                                          P, P, P, P, SZ, P, P]
         lib.mi_debug_wait_failure.argtypes = [P]
         lib.mi_vs_index_static.argtypes = [P, P, I, I, I, I, F, I, I, I, P, I, P, P, P, P, P]
+        lib.mi_dense_attn.argtypes = [P, P, P, I, I, I, I, F, P, I, P, P, P, P, SZ, P]
         for name in EXPORTS[5:]:
             getattr(lib, name).restype = I
         _lib = lib
@@ -258,6 +260,19 @@ def mi_ashape_attn(q, k, v, sink, window, heads=None, scale=0.0, out=None, lse=N
                                       window, hp, n, _ptr(out), _ptr(lse), _ptr(err_count), None,
                                       0, _stream(stream))
     _check("mi_ashape_attn", rc)
+    return out, lse
+
+
+def mi_dense_attn(q, k, v, heads=None, scale=0.0, out=None, lse=None, want_lse=True,
+                  err_count=None, stream=None):
+    """Dense causal attention (every key j <= i) on the same engine."""
+    Hq, Hkv, N, d = _shape(q, k)
+    harr, n, hp = _heads(heads, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse)
+    rc = _lib_handle().mi_dense_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, hp, n,
+                                     _ptr(out), _ptr(lse), _ptr(err_count), None, 0,
+                                     _stream(stream))
+    _check("mi_dense_attn", rc)
     return out, lse
 
 

@@ -138,7 +138,8 @@ size_t mi_workspace_bytes(int op, int Hq, int Hkv, int N, int d, int n_heads, in
         case MI_OP_BS_INDEX: return bs_index_bytes(n, Hkv, N, d);
         case MI_OP_VS_ATTN: return vs_prep_bytes(n, N, vertical_size > 0 ? vertical_size : 1);
         case MI_OP_BS_ATTN:
-        case MI_OP_ASHAPE_ATTN: return 256;
+        case MI_OP_ASHAPE_ATTN:
+        case MI_OP_DENSE_ATTN: return 256;
         default: return 0;
     }
     (void)slash_size;
@@ -292,6 +293,23 @@ int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq,
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
+int mi_dense_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
+                  int d, float scale, const int32_t* heads, int n_heads, mi_bf16* out,
+                  float* lse, int32_t* err_count, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    HeadList hl;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
+    if (rc) return rc;
+    if (!v || !out) return MI_ERR_INVALID_ARG;
+    if (hl.n == 0) return MI_OK;
+    AttnLaunch a;
+    attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
+    set_pattern(hl, MI_PATTERN_DENSE);
+    a.heads = hl;
+    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
 int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
                      int N, int d, float scale, const int8_t* pattern, const mi_params* p,
                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
@@ -305,6 +323,7 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
     for (int h = 0; h < Hq; ++h) {
         switch (pattern[h]) {
             case MI_PATTERN_ASHAPE: all.e[h] = pack_head(h, MI_PATTERN_ASHAPE, n_a++); break;
+            case MI_PATTERN_DENSE: all.e[h] = pack_head(h, MI_PATTERN_DENSE, 0); break;
             case MI_PATTERN_VS:
                 all.e[h] = pack_head(h, MI_PATTERN_VS, vs.n);
                 vs.e[vs.n] = pack_head(h, MI_PATTERN_VS, vs.n);

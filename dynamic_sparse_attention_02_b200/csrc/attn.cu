@@ -5,7 +5,8 @@
 // causal flash-style attention with an online softmax over only its selected
 // keys: the sink plus local band (A-shape), the chosen 64x64 blocks
 // (Block-Sparse), or the gathered vertical columns plus the 64x64 tiles its
-// slash diagonals touch (Vertical-Slash), without counting a key twice.
+// slash diagonals touch (Vertical-Slash), without counting a key twice.  A
+// dense head (every causal key) runs on the same engine.
 //
 // Work item = one query head x one 256-row "super tile" (four 64-row query
 // blocks), held as two 128-row slots.  The producer enumerates the item's
@@ -500,6 +501,9 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
                 }
             } else if (pattern == MI_PATTERN_BS) {
                 m = (patmap[b >> 3] >> ((b & 7) * 4)) & 0xF;
+            } else if (pattern == MI_PATTERN_DENSE) {
+                for (int qq = 0; qq < nqb; ++qq)  // every causal block
+                    if (b <= qb0 + qq) m |= 1 << qq;
             } else {
                 for (int qq = 0; qq < nqb; ++qq) {
                     const int qb = qb0 + qq;

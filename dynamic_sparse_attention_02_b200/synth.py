@@ -34,6 +34,7 @@ import torch
 PATTERN_ASHAPE = 0
 PATTERN_VS = 1
 PATTERN_BS = 2
+PATTERN_DENSE = 3
 
 ROPE_THETA = 500000.0
 SEED_BASE = 20260000

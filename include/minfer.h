@@ -64,14 +64,18 @@ enum {
     MI_ERR_CUDA = 4         /* a CUDA call failed; see mi_last_cuda_error() */
 };
 
-enum { MI_PATTERN_ASHAPE = 0, MI_PATTERN_VS = 1, MI_PATTERN_BS = 2 };
+/* Per-head patterns of the router.  DENSE is plain causal attention over every
+ * key j <= i: the prefill MInference is measured against (guide, "Prefill
+ * Latency Benchmark"), and the choice for a head no sparse pattern fits. */
+enum { MI_PATTERN_ASHAPE = 0, MI_PATTERN_VS = 1, MI_PATTERN_BS = 2, MI_PATTERN_DENSE = 3 };
 
 enum {
     MI_OP_VS_INDEX = 1,
     MI_OP_BS_INDEX = 2,
     MI_OP_VS_ATTN = 3,
     MI_OP_BS_ATTN = 4,
-    MI_OP_ASHAPE_ATTN = 5
+    MI_OP_ASHAPE_ATTN = 5,
+    MI_OP_DENSE_ATTN = 6
 };
 
 #define MI_MAX_HEADS 256
@@ -198,6 +202,15 @@ int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq,
                    int d, float scale, int sink, int window, const int32_t* heads, int n_heads,
                    mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
                    void* stream);
+
+/*
+ * Dense causal attention: row i attends every key j <= i, on the same engine
+ * as the sparse entry points (every causal 64x64 tile computed).  No
+ * workspace is needed (ws may be NULL).  out / lse as for mi_vs_sparse_attn.
+ */
+int mi_dense_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
+                  int d, float scale, const int32_t* heads, int n_heads, mi_bf16* out,
+                  float* lse, int32_t* err_count, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * One attention layer with a per-head pattern table (guide, "Phase 2: The

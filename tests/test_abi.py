@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = header_functions()
-    assert len(names) == 13
+    assert len(names) == 14
     assert sorted(B.EXPORTS) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -90,6 +90,11 @@ def test_attention_validation(lib):
                               0, None) == B.MI_ERR_INVALID_ARG
     assert lib.mi_ashape_attn(f, f, f, 4, 2, 520, 128, 0.0, 4, 8, None, 0, f, None, None, None,
                               0, None) == B.MI_ERR_UNSUPPORTED
+    # dense: v and out required, same shape rules
+    assert lib.mi_dense_attn(f, f, None, 4, 2, 512, 128, 0.0, None, 0, f, None, None, None, 0,
+                             None) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_dense_attn(f, f, f, 4, 2, 520, 128, 0.0, None, 0, f, None, None, None, 0,
+                             None) == B.MI_ERR_UNSUPPORTED
     # VS attention: workspace
     assert lib.mi_vs_sparse_attn(f, f, f, 4, 2, 512, 128, 0.0, f, 8, f, 8, None, 0, f, None,
                                  None, f, 8, None) == B.MI_ERR_WORKSPACE
@@ -105,7 +110,7 @@ def test_prefill_layer_validation(lib):
     assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, bad.ctypes.data_as(ctypes.c_void_p),
                                 ctypes.byref(p), f, None, None, f, 1 << 30, None,
                                 None) == B.MI_ERR_INVALID_ARG
-    good = np.array([0, 1, 2, 1], np.int8)
+    good = np.array([0, 1, 2, 3], np.int8)  # A-shape, VS, BS, dense
     assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, good.ctypes.data_as(ctypes.c_void_p),
                                 ctypes.byref(p), f, None, None, f, 16, None,
                                 None) == B.MI_ERR_WORKSPACE

@@ -148,6 +148,20 @@ def test_vs_attn_matches_oracle(Hq, Hkv, N, d, L, kv, ks):
         check_attn(out[h], lse[h], *refs[h], what=f"vs h{h}")
 
 
+@pytest.mark.parametrize("Hq,Hkv,N,d", [
+    (4, 1, 1088, 128),   # GQA 4:1, ragged tail
+    (2, 2, 576, 64),
+    (1, 1, 64, 128),     # one block
+])
+def test_dense_attn_matches_oracle(Hq, Hkv, N, d):
+    q, k, v = rand_bf16(Hq, Hkv, N, d, 31)
+    out, lse = B.mi_dense_attn(q, k, v)
+    torch.cuda.synchronize()
+    for h in range(Hq):
+        qs, ks_, vs_ = head_slices(q, k, v, h)
+        check_attn(out[h], lse[h], *oracle.attn_dense(qs, ks_, vs_, 0), what=f"dense h{h}")
+
+
 def test_vs_attn_unsorted_duplicates_and_empty_rows():
     """Unsorted, repeated index entries count once; rows before every key are empty."""
     q, k, v = rand_bf16(2, 1, 512, 128, 13)
@@ -222,10 +236,10 @@ def test_full_budgets_equal_dense_sdpa():
 
 @pytest.mark.parametrize("N,d", [(1024, 128), (576, 64)])
 def test_prefill_layer_mixed_matches_oracle(N, d):
-    """The pattern router: mixed A-shape / VS / BS heads in one launch."""
+    """The pattern router: mixed A-shape / VS / BS / dense heads in one launch."""
     w = synth.workload("mixed_n256k_llama3_8b", Hq=8, Hkv=2, N=N, d=d)
     x = synth.make_inputs(w, device="cuda")
-    pattern = np.array([0, 1, 2, 1, 2, 0, 1, 2], np.int8)
+    pattern = np.array([0, 1, 2, 3, 2, 0, 1, 3], np.int8)
     p = B.make_params(last_q=64, vertical_size=40, slash_size=60, topk_blocks=4, sink=64,
                       window=256)
     out, lse = B.mi_prefill_layer(x["q"], x["k"], x["v"], pattern, p, want_lse=True)
@@ -237,6 +251,8 @@ def test_prefill_layer_mixed_matches_oracle(N, d):
         elif pattern[h] == 1:
             a, b, _, _ = oracle.vs_index(qs, ks_, 0, 64, 40, 60)
             ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, a, b)
+        elif pattern[h] == 3:
+            ro, rl = oracle.attn_dense(qs, ks_, vs_, 0)
         else:
             bi, bc = oracle.bs_index(qs, ks_, 0, 4)
             ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi, bc)
