@@ -61,6 +61,8 @@ def parse_args(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override N of the workload (smaller profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense-prefill comparison (every head dense causal)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0,
                     help="approximate CPU seconds for the oracle baseline sample")
@@ -429,6 +431,29 @@ def run_minfer(args):
                "d2h_bytes_per_step": int(hout.numel() * 2), "steps": n_e2e}
         assert torch.equal(hout, out.cpu()), "e2e output differs from the device output"
 
+    # The pages' headline comparison: the same layer with every head dense
+    # causal (the prefill MInference is measured against), on the same engine.
+    dense = None
+    if not args.no_dense:
+        dout = torch.empty_like(out)
+        n_dense = 1 if w.N > 262144 else max(1, min(args.steps, 3))
+        B.mi_dense_attn(q, k, v, out=dout, want_lse=False)
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n_dense):
+            B.mi_dense_attn(q, k, v, out=dout, want_lse=False)
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms_dense = max_over_ranks(a.elapsed_time(b) / n_dense)
+        log(f"dense causal attention {ms_dense:.2f} ms")
+        dense = {"ms": ms_dense, "steps": n_dense,
+                 "speedup_vs_dense": ms_dense / ms_step_max,
+                 "tflops": 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq / (ms_dense * 1e-3) / 1e12}
+        del dout
+
     # algorithmic work of the attention launch (from this layer's own index)
     useful = 0.0
     tiles = 0
@@ -489,6 +514,7 @@ def run_minfer(args):
                          "flops_per_launch": useful},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "dense_prefill": dense,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
