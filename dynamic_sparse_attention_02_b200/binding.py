@@ -32,7 +32,8 @@ MI_BLOCK = 64
 EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
            "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
-           "mi_vs_index_static", "mi_dense_attn"]
+           "mi_vs_index_static", "mi_dense_attn", "mi_prefill_workspace_bytes_heads",
+           "mi_prefill_layer_heads"]
 
 
 class MinferError(RuntimeError):
@@ -81,8 +82,13 @@ def _lib_handle():
         lib.mi_debug_wait_failure.argtypes = [P]
         lib.mi_vs_index_static.argtypes = [P, P, I, I, I, I, F, I, I, I, P, I, P, P, P, P, P]
         lib.mi_dense_attn.argtypes = [P, P, P, I, I, I, I, F, P, I, P, P, P, P, SZ, P]
+        lib.mi_prefill_workspace_bytes_heads.argtypes = [I, I, I, I, P, P]
+        lib.mi_prefill_workspace_bytes_heads.restype = SZ
+        lib.mi_prefill_layer_heads.argtypes = [P, P, P, I, I, I, I, F, P, P, P, P, P, P, SZ, P,
+                                               P]
         for name in EXPORTS[5:]:
-            getattr(lib, name).restype = I
+            if name != "mi_prefill_workspace_bytes_heads":
+                getattr(lib, name).restype = I
         _lib = lib
     return _lib
 
@@ -158,6 +164,19 @@ def mi_prefill_workspace_bytes(Hq, Hkv, N, d, pattern, params: mi_params) -> int
     pat = None if pattern is None else np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
     pp = None if pat is None else pat.ctypes.data_as(ctypes.c_void_p)
     return int(_lib_handle().mi_prefill_workspace_bytes(Hq, Hkv, N, d, pp, ctypes.byref(params)))
+
+
+def _params_array(params):
+    arr = (mi_params * len(params))(*params)
+    return arr
+
+
+def mi_prefill_workspace_bytes_heads(Hq, Hkv, N, d, pattern, params) -> int:
+    """Workspace of mi_prefill_layer_heads: `params` holds one mi_params per head."""
+    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
+    arr = _params_array(params)
+    return int(_lib_handle().mi_prefill_workspace_bytes_heads(
+        Hq, Hkv, N, d, pat.ctypes.data_as(ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p)))
 
 
 def mi_vs_index(q, k, last_q, vertical_size, slash_size, heads: Optional[Sequence[int]] = None,
@@ -273,6 +292,25 @@ def mi_dense_attn(q, k, v, heads=None, scale=0.0, out=None, lse=None, want_lse=T
                                      _ptr(out), _ptr(lse), _ptr(err_count), None, 0,
                                      _stream(stream))
     _check("mi_dense_attn", rc)
+    return out, lse
+
+
+def mi_prefill_layer_heads(q, k, v, pattern, params, scale=0.0, out=None, lse=None,
+                           want_lse=False, err_count=None, ws=None, stream=None):
+    """One layer with one mi_params per head (host int8 pattern [Hq], params [Hq])."""
+    Hq, Hkv, N, d = _shape(q, k)
+    if len(params) != Hq:
+        raise ValueError("one mi_params per query head")
+    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
+    arr = _params_array(params)
+    out, lse = _attn_out(q, out, lse, want_lse)
+    need = mi_prefill_workspace_bytes_heads(Hq, Hkv, N, d, pat, params)
+    ws = _workspace(need, q.device, ws)
+    rc = _lib_handle().mi_prefill_layer_heads(
+        _ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, pat.ctypes.data_as(ctypes.c_void_p),
+        ctypes.cast(arr, ctypes.c_void_p), _ptr(out), _ptr(lse), _ptr(err_count), _ptr(ws),
+        ws.numel(), _stream(stream), None)
+    _check("mi_prefill_layer_heads", rc)
     return out, lse
 
 

@@ -310,46 +310,88 @@ int mi_dense_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, 
     return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
-int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
-                     int N, int d, float scale, const int8_t* pattern, const mi_params* p,
-                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
-                     void* stream, void* const* stage_events) {
-    HeadList all;
-    int rc = check_shapes(q, k, Hq, Hkv, N, d, nullptr, 0, all);
-    if (rc) return rc;
-    if (!v || !out || !pattern || !p) return MI_ERR_INVALID_ARG;
-    HeadList vs{}, bs{};
+namespace {
+
+// One layer with either one parameter set for every head (per_head = false)
+// or one per head.  VS heads must share last_q (the score passes take one row
+// count); budgets, block counts, sink and window may differ per head.
+struct LayerPlan {
+    HeadList all, vs, bs;
     int n_a = 0;
+    mi_params pp{};  // layer-wide maxima: buffer sizes and index row strides
+    int32_t kv_h[MI_MAX_HEADS], ks_h[MI_MAX_HEADS], tk_h[MI_MAX_HEADS];
+    int32_t sink_h[MI_MAX_HEADS], win_h[MI_MAX_HEADS];
+};
+
+int plan_layer(int Hq, int N, const int8_t* pattern, const mi_params* params, bool per_head,
+               LayerPlan& lp) {
+    lp.vs.n = lp.bs.n = 0;
+    lp.n_a = 0;
+    int L = -1, kv_max = 0, ks_max = 0, tk_max = 0;
     for (int h = 0; h < Hq; ++h) {
+        const mi_params& ph = params[per_head ? h : 0];
         switch (pattern[h]) {
-            case MI_PATTERN_ASHAPE: all.e[h] = pack_head(h, MI_PATTERN_ASHAPE, n_a++); break;
-            case MI_PATTERN_DENSE: all.e[h] = pack_head(h, MI_PATTERN_DENSE, 0); break;
-            case MI_PATTERN_VS:
-                all.e[h] = pack_head(h, MI_PATTERN_VS, vs.n);
-                vs.e[vs.n] = pack_head(h, MI_PATTERN_VS, vs.n);
-                ++vs.n;
+            case MI_PATTERN_ASHAPE:
+                if (ph.sink < 0 || ph.window < 1) return MI_ERR_INVALID_ARG;
+                lp.sink_h[lp.n_a] = ph.sink;
+                lp.win_h[lp.n_a] = ph.window;
+                lp.all.e[h] = pack_head(h, MI_PATTERN_ASHAPE, lp.n_a++);
                 break;
-            case MI_PATTERN_BS:
-                all.e[h] = pack_head(h, MI_PATTERN_BS, bs.n);
-                bs.e[bs.n] = pack_head(h, MI_PATTERN_BS, bs.n);
-                ++bs.n;
+            case MI_PATTERN_DENSE: lp.all.e[h] = pack_head(h, MI_PATTERN_DENSE, 0); break;
+            case MI_PATTERN_VS: {
+                if (L >= 0 && ph.last_q != L) return MI_ERR_INVALID_ARG;
+                L = ph.last_q;
+                const int rc = check_vs_params(N, ph.last_q, ph.vertical_size, ph.slash_size);
+                if (rc) return rc;
+                const int kv = ph.vertical_size < N ? ph.vertical_size : N;
+                const int ks = ph.slash_size < N ? ph.slash_size : N;
+                lp.kv_h[lp.vs.n] = kv;
+                lp.ks_h[lp.vs.n] = ks;
+                kv_max = kv > kv_max ? kv : kv_max;
+                ks_max = ks > ks_max ? ks : ks_max;
+                lp.all.e[h] = pack_head(h, MI_PATTERN_VS, lp.vs.n);
+                lp.vs.e[lp.vs.n] = pack_head(h, MI_PATTERN_VS, lp.vs.n);
+                ++lp.vs.n;
                 break;
+            }
+            case MI_PATTERN_BS: {
+                if (ph.topk_blocks < 0) return MI_ERR_INVALID_ARG;
+                const int nB = N / MI_BLOCK;
+                const int tk = ph.topk_blocks < nB ? ph.topk_blocks : nB;
+                lp.tk_h[lp.bs.n] = tk;
+                tk_max = tk > tk_max ? tk : tk_max;
+                lp.all.e[h] = pack_head(h, MI_PATTERN_BS, lp.bs.n);
+                lp.bs.e[lp.bs.n] = pack_head(h, MI_PATTERN_BS, lp.bs.n);
+                ++lp.bs.n;
+                break;
+            }
             default: return MI_ERR_INVALID_ARG;
         }
     }
-    if (vs.n && (rc = check_vs_params(N, p->last_q, p->vertical_size, p->slash_size))) return rc;
-    if (bs.n && p->topk_blocks < 0) return MI_ERR_INVALID_ARG;
-    if (n_a && (p->sink < 0 || p->window < 1)) return MI_ERR_INVALID_ARG;
-    mi_params pp = *p;
-    if (!vs.n) pp.vertical_size = pp.slash_size = 0;
-    if (!bs.n) pp.topk_blocks = 0;
-    if (vs.n && pp.vertical_size < 1) pp.vertical_size = 1;  // keep carved buffers non-empty
+    lp.pp = params[0];
+    lp.pp.last_q = L > 0 ? L : params[0].last_q;
+    lp.pp.vertical_size = lp.vs.n ? (kv_max > 0 ? kv_max : 1) : 0;  // carved buffers non-empty
+    lp.pp.slash_size = lp.vs.n ? ks_max : 0;
+    lp.pp.topk_blocks = lp.bs.n ? tk_max : 0;
+    return MI_OK;
+}
+
+int prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
+                  int d, float scale, const int8_t* pattern, const mi_params* params,
+                  bool per_head, mi_bf16* out, float* lse, int32_t* err_count, void* ws,
+                  size_t ws_bytes, void* stream, void* const* stage_events) {
+    LayerPlan lp;
+    int rc = check_shapes(q, k, Hq, Hkv, N, d, nullptr, 0, lp.all);
+    if (rc) return rc;
+    if (!v || !out || !pattern || !params) return MI_ERR_INVALID_ARG;
+    if ((rc = plan_layer(Hq, N, pattern, params, per_head, lp))) return rc;
+    const mi_params& pp = lp.pp;
     WsCarver sizer(nullptr);
-    carve_layer(sizer, vs.n, bs.n, Hkv, N, d, pp);
+    carve_layer(sizer, lp.vs.n, lp.bs.n, Hkv, N, d, pp);
     if ((rc = check_ws(ws, ws_bytes, sizer.bytes()))) return rc;
 
     WsCarver c(ws);
-    LayerWs w = carve_layer(c, vs.n, bs.n, Hkv, N, d, pp);
+    LayerWs w = carve_layer(c, lp.vs.n, lp.bs.n, Hkv, N, d, pp);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const double sc = eff_scale(scale, d);
     auto rec = [&](int i) -> int {
@@ -359,28 +401,30 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
     if ((rc = rec(MI_STAGE_START))) return rc;
     const bf16* qb = reinterpret_cast<const bf16*>(q);
     const bf16* kb = reinterpret_cast<const bf16*>(k);
-    if (vs.n) {
+    if (lp.vs.n) {
         rc = cuda_status(launch_vs_index(qb, kb, Hq, Hkv, N, d, sc, pp.last_q, pp.vertical_size,
-                                         pp.slash_size, vs, w.v_idx, w.s_idx, nullptr, nullptr,
-                                         w.vsi, st));
+                                         pp.slash_size, lp.vs, w.v_idx, w.s_idx, nullptr,
+                                         nullptr, w.vsi, st, per_head ? lp.kv_h : nullptr,
+                                         per_head ? lp.ks_h : nullptr));
         if (rc) return rc;
     }
-    if (bs.n) {
-        rc = cuda_status(launch_bs_index(qb, kb, Hq, Hkv, N, d, sc, pp.topk_blocks, bs, w.blk_idx,
-                                         w.blk_cnt, w.bsi, st));
+    if (lp.bs.n) {
+        rc = cuda_status(launch_bs_index(qb, kb, Hq, Hkv, N, d, sc, pp.topk_blocks, lp.bs,
+                                         w.blk_idx, w.blk_cnt, w.bsi, st,
+                                         per_head ? lp.tk_h : nullptr));
         if (rc) return rc;
     }
     if ((rc = rec(MI_STAGE_INDEX_DONE))) return rc;
-    if (vs.n) {
+    if (lp.vs.n) {
         rc = cuda_status(launch_vs_prep(w.v_idx, pp.vertical_size, pp.vertical_size, w.s_idx,
-                                        pp.slash_size, pp.slash_size, N, vs.n, w.prep, err_count,
-                                        st));
+                                        pp.slash_size, pp.slash_size, N, lp.vs.n, w.prep,
+                                        err_count, st));
         if (rc) return rc;
     }
     if ((rc = rec(MI_STAGE_PREP_DONE))) return rc;
     AttnLaunch a;
     attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
-    a.heads = all;
+    a.heads = lp.all;
     a.dbits = w.prep.dbits;
     a.vlist = w.prep.vlist;
     a.vcnt = w.prep.vcnt;
@@ -390,8 +434,42 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
     a.topk = pp.topk_blocks;
     a.sink = pp.sink;
     a.window = pp.window;
+    a.sink_h = lp.sink_h;
+    a.window_h = lp.win_h;
+    a.n_asw = lp.n_a;
     if ((rc = cuda_status(launch_sparse_attn(a, st)))) return rc;
     return rec(MI_STAGE_ATTN_DONE);
+}
+
+}  // namespace
+
+int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                     int N, int d, float scale, const int8_t* pattern, const mi_params* p,
+                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                     void* stream, void* const* stage_events) {
+    return prefill_layer(q, k, v, Hq, Hkv, N, d, scale, pattern, p, false, out, lse, err_count,
+                         ws, ws_bytes, stream, stage_events);
+}
+
+size_t mi_prefill_workspace_bytes_heads(int Hq, int Hkv, int N, int d, const int8_t* pattern,
+                                        const mi_params* params) {
+    if (!pattern || !params || Hq <= 0 || Hq > MI_MAX_HEADS || Hkv <= 0 || N <= 0 ||
+        N % MI_BLOCK || (d != 64 && d != 128))
+        return 0;
+    LayerPlan lp;
+    if (plan_layer(Hq, N, pattern, params, true, lp) != MI_OK) return 0;
+    WsCarver c(nullptr);
+    carve_layer(c, lp.vs.n, lp.bs.n, Hkv, N, d, lp.pp);
+    return c.bytes();
+}
+
+int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq,
+                           int Hkv, int N, int d, float scale, const int8_t* pattern,
+                           const mi_params* params, mi_bf16* out, float* lse,
+                           int32_t* err_count, void* ws, size_t ws_bytes, void* stream,
+                           void* const* stage_events) {
+    return prefill_layer(q, k, v, Hq, Hkv, N, d, scale, pattern, params, true, out, lse,
+                         err_count, ws, ws_bytes, stream, stage_events);
 }
 
 int mi_debug_wait_failure(int32_t* record8) {

@@ -125,7 +125,7 @@ struct AttnParams {
     const int32_t* blk_idx;
     const int32_t* blk_cnt;
     int topk;
-    int sink, window;
+    int2 asw[MI_MAX_HEADS];  // A-shape heads, by A-shape position: (sink, window)
     int32_t* err;
     HeadList heads;  // sorted by KV head
     int ngroups;     // KV heads present in `heads`
@@ -507,7 +507,7 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
             } else {
                 for (int qq = 0; qq < nqb; ++qq) {
                     const int qb = qb0 + qq;
-                    if (b <= qb && (64 * b < p.sink || 64 * (qb - b) - 63 < p.window))
+                    if (b <= qb && (64 * b < p.asw[pidx].x || 64 * (qb - b) - 63 < p.asw[pidx].y))
                         m |= 1 << qq;
                 }
             }
@@ -729,6 +729,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     const uint32_t e = p.heads.e[pos];
     const int qh = head_qh(e), pattern = head_pattern(e);
     const bool ashape = pattern == MI_PATTERN_ASHAPE;
+    const int sink = p.asw[head_pidx(e)].x, window = p.asw[head_pidx(e)].y;  // A-shape only
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     // warp-uniform TMEM address (tcgen05.ld/st take it from a uniform register)
     const uint32_t tSlot = __shfl_sync(0xffffffffu, tmem + 256 * x + lane_off, 0);
@@ -763,7 +764,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                     const long long j0 = 64LL * d.b;
                     keep = low_bits(i - j0 + 1);  // causal: columns <= i
                     if (ashape)  // sink (j < sink) or local window (i - j < window)
-                        keep &= low_bits(p.sink - j0) | ~low_bits(i - j0 - p.window + 1);
+                        keep &= low_bits(sink - j0) | ~low_bits(i - j0 - window + 1);
                 }
             } else {
                 // gathered columns ascend: those <= i form a prefix
@@ -1151,8 +1152,9 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
     p.blk_idx = a.blk_idx;
     p.blk_cnt = a.blk_cnt;
     p.topk = a.topk;
-    p.sink = a.sink;
-    p.window = a.window;
+    for (int i = 0; i < MI_MAX_HEADS; ++i)
+        p.asw[i] = make_int2(a.sink_h && i < a.n_asw ? a.sink_h[i] : a.sink,
+                             a.window_h && i < a.n_asw ? a.window_h[i] : a.window);
     p.err = a.err_count;
     // heads sorted by KV head (stable); each entry keeps its own per-pattern position
     p.heads.n = 0;

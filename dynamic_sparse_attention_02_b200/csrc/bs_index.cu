@@ -80,7 +80,7 @@ constexpr size_t bs_fixed_smem() {
 template <int D>
 __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     const float* __restrict__ qm, const float* __restrict__ km, int Hq, int Hkv, int nB,
-    int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk,
+    int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk, RowCounts tk,
     int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt) {
     extern __shared__ __align__(16) double dsm[];
     double* Qs = dsm;                          // [D][kMaxR]
@@ -143,10 +143,11 @@ __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     }
     __syncthreads();
 
+    const int budget = pos < tk.n ? tk.k[pos] : topk;  // this head's budget (row stride: topk)
     for (int r = warp; r < nr; r += kTopkThreads / 32) {
         const int bq = bq0 + r;
         const int n = bq + 1;
-        const int kk = min(topk, n);
+        const int kk = min(budget, n);
         int32_t* o = blk_idx + ((size_t)pos * nB + bq) * topk;
         for (int t = kk + lane; t < topk; t += 32) o[t] = -1;
         if (lane == 0) blk_cnt[(size_t)pos * nB + bq] = kk;
@@ -175,7 +176,7 @@ int rows_per_cta(int nB) {
 template <int D>
 cudaError_t launch_bs_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, double scale,
                         int topk, const HeadList& heads, int32_t* blk_idx, int32_t* blk_cnt,
-                        const BsIndexWs& ws, cudaStream_t st) {
+                        const BsIndexWs& ws, cudaStream_t st, const int32_t* topk_rows) {
     const int nB = N / 64;
     // KV heads used by the listed query heads, each once
     HeadList kvs{};
@@ -185,13 +186,18 @@ cudaError_t launch_bs_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, do
         if (used[g]) kvs.e[kvs.n++] = pack_head(g, 0, 0);
     meanpool_kernel<D><<<dim3(nB, heads.n), kPoolThreads, 0, st>>>(q, N, nB, heads, ws.qm);
     meanpool_kernel<D><<<dim3(nB, kvs.n), kPoolThreads, 0, st>>>(k, N, nB, kvs, ws.km);
+    RowCounts tk{};
+    if (topk_rows) {
+        tk.n = heads.n;
+        for (int i = 0; i < heads.n; ++i) tk.k[i] = topk_rows[i];
+    }
     const int R = rows_per_cta<D>(nB);
     const size_t smem = bs_fixed_smem<D>() + (size_t)R * (nB + R) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bs_topk_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bs_topk_kernel<D><<<dim3((nB + R - 1) / R, heads.n), kTopkThreads, smem, st>>>(
-        ws.qm, ws.km, Hq, Hkv, nB, kvs.n, heads, kvs, R, scale, topk, blk_idx, blk_cnt);
+        ws.qm, ws.km, Hq, Hkv, nB, kvs.n, heads, kvs, R, scale, topk, tk, blk_idx, blk_cnt);
     return cudaGetLastError();
 }
 
@@ -207,11 +213,14 @@ BsIndexWs carve_bs_index(WsCarver& c, int n_heads, int Hkv, int N, int d) {
 
 cudaError_t launch_bs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
                             double scale, int topk, const HeadList& heads, int32_t* blk_idx,
-                            int32_t* blk_cnt, const BsIndexWs& ws, cudaStream_t st) {
+                            int32_t* blk_cnt, const BsIndexWs& ws, cudaStream_t st,
+                            const int32_t* topk_rows) {
     if (heads.n == 0) return cudaSuccess;
     if (d == 128)
-        return launch_bs_d<128>(q, k, Hq, Hkv, N, scale, topk, heads, blk_idx, blk_cnt, ws, st);
-    return launch_bs_d<64>(q, k, Hq, Hkv, N, scale, topk, heads, blk_idx, blk_cnt, ws, st);
+        return launch_bs_d<128>(q, k, Hq, Hkv, N, scale, topk, heads, blk_idx, blk_cnt, ws, st,
+                                topk_rows);
+    return launch_bs_d<64>(q, k, Hq, Hkv, N, scale, topk, heads, blk_idx, blk_cnt, ws, st,
+                           topk_rows);
 }
 
 }  // namespace minfer

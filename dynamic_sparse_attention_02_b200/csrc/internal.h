@@ -31,6 +31,13 @@ __host__ __device__ inline int kv_head_of(int qh, int Hq, int Hkv) {
     return (int)(((long long)qh * Hkv) / Hq);
 }
 
+// One count per row of a batched top-k (per-head budgets); rows past `n` and
+// a null list fall back to the launch's single budget.
+struct RowCounts {
+    int n;
+    int32_t k[MI_MAX_HEADS];
+};
+
 // Bump allocator over the caller's workspace.  With base == nullptr it only
 // measures, so size queries and launches carve identically.
 struct WsCarver {
@@ -60,10 +67,13 @@ struct VsIndexWs {
 };
 VsIndexWs carve_vs_index(WsCarver& c, int n_heads, int N, int L, bool need_vscore,
                          bool need_sscore);
+// kv / ks: budgets and index row strides; kv_rows / ks_rows (optional, host,
+// one per listed head, each <= kv / ks): per-head budgets, -1 past them.
 cudaError_t launch_vs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
                             double scale, int L, int kv, int ks, const HeadList& heads,
                             int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
-                            const VsIndexWs& ws, cudaStream_t st);
+                            const VsIndexWs& ws, cudaStream_t st,
+                            const int32_t* kv_rows = nullptr, const int32_t* ks_rows = nullptr);
 
 // ----------------------------------------------------------- BS index
 struct BsIndexWs {
@@ -71,9 +81,12 @@ struct BsIndexWs {
     float* km;  // [Hkv][nB][d]
 };
 BsIndexWs carve_bs_index(WsCarver& c, int n_heads, int Hkv, int N, int d);
+// topk: budget and index row stride; topk_rows (optional, host, one per listed
+// head, each <= topk): per-head budgets.
 cudaError_t launch_bs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
                             double scale, int topk, const HeadList& heads, int32_t* blk_idx,
-                            int32_t* blk_cnt, const BsIndexWs& ws, cudaStream_t st);
+                            int32_t* blk_cnt, const BsIndexWs& ws, cudaStream_t st,
+                            const int32_t* topk_rows = nullptr);
 
 // ----------------------------------------------------------- attention
 struct VsPrepWs {
@@ -104,8 +117,12 @@ struct AttnLaunch {
     const int32_t* blk_idx;
     const int32_t* blk_cnt;
     int topk;
-    // A-shape
+    // A-shape (sink_h / window_h, optional host arrays indexed by the head's
+    // A-shape position, override sink / window per head)
     int sink, window;
+    const int32_t* sink_h;
+    const int32_t* window_h;
+    int n_asw;  // entries in sink_h / window_h
     int32_t* err_count;
 };
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);

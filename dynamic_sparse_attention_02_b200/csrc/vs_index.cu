@@ -317,11 +317,11 @@ struct GlobalKeys {
 // Top-k of each row of scores [rows][n]; out row stride out_stride, -1 past k.
 __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict__ scores,
                                                          int n, int k, int32_t* out,
-                                                         int out_stride) {
+                                                         int out_stride, RowCounts rk) {
     __shared__ TopkSmem s;
     const int row = blockIdx.x;
     int32_t* o = out + (size_t)row * out_stride;
-    const int kk = min(k, n);
+    const int kk = min(row < rk.n ? rk.k[row] : k, n);
     for (int t = kk + threadIdx.x; t < out_stride; t += blockDim.x) o[t] = -1;
     if (kk <= 0) return;
     if (kk == n) {
@@ -349,7 +349,7 @@ template <int D>
 cudaError_t launch_vs_index_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, double scale,
                               int L, int kv, int ks, const HeadList& heads, int32_t* v_idx,
                               int32_t* s_idx, float* vsc, float* ssc, const VsIndexWs& ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, const int32_t* kv_rows, const int32_t* ks_rows) {
     const int n = heads.n;
     const int nchunks = (N + kVsChunk - 1) / kVsChunk;
     const int nrt = (L + 63) / 64;
@@ -367,8 +367,17 @@ cudaError_t launch_vs_index_d(const bf16* q, const bf16* k, int Hq, int Hkv, int
     vs_rowmerge_kernel<<<n, 64, 0, st>>>(ws.m_part, ws.l_part, L, nchunks, ws.mrow, ws.linv);
     vs_colslash_kernel<D><<<dim3(nchunks, n), kThreads, sm2, st>>>(
         q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.mrow, ws.linv, vsc, ssc);
-    topk_rows_kernel<<<n, 1024, 0, st>>>(vsc, N, kv, v_idx, kv);
-    topk_rows_kernel<<<n, 1024, 0, st>>>(ssc, N, ks, s_idx, ks);
+    RowCounts rv{}, rs{};
+    if (kv_rows) {
+        rv.n = n;
+        for (int i = 0; i < n; ++i) rv.k[i] = kv_rows[i];
+    }
+    if (ks_rows) {
+        rs.n = n;
+        for (int i = 0; i < n; ++i) rs.k[i] = ks_rows[i];
+    }
+    topk_rows_kernel<<<n, 1024, 0, st>>>(vsc, N, kv, v_idx, kv, rv);
+    topk_rows_kernel<<<n, 1024, 0, st>>>(ssc, N, ks, s_idx, ks, rs);
     return cudaGetLastError();
 }
 
@@ -390,15 +399,16 @@ VsIndexWs carve_vs_index(WsCarver& c, int n_heads, int N, int L, bool need_vscor
 cudaError_t launch_vs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N, int d,
                             double scale, int L, int kv, int ks, const HeadList& heads,
                             int32_t* v_idx, int32_t* s_idx, float* v_score, float* s_score,
-                            const VsIndexWs& ws, cudaStream_t st) {
+                            const VsIndexWs& ws, cudaStream_t st, const int32_t* kv_rows,
+                            const int32_t* ks_rows) {
     if (heads.n == 0) return cudaSuccess;
     float* vsc = v_score ? v_score : ws.vscore;
     float* ssc = s_score ? s_score : ws.sscore;
     if (d == 128)
         return launch_vs_index_d<128>(q, k, Hq, Hkv, N, scale, L, kv, ks, heads, v_idx, s_idx,
-                                      vsc, ssc, ws, st);
+                                      vsc, ssc, ws, st, kv_rows, ks_rows);
     return launch_vs_index_d<64>(q, k, Hq, Hkv, N, scale, L, kv, ks, heads, v_idx, s_idx, vsc,
-                                 ssc, ws, st);
+                                 ssc, ws, st, kv_rows, ks_rows);
 }
 
 }  // namespace minfer

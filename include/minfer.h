@@ -65,8 +65,10 @@ enum {
 };
 
 /* Per-head patterns of the router.  DENSE is plain causal attention over every
- * key j <= i: the prefill MInference is measured against (guide, "Prefill
- * Latency Benchmark"), and the choice for a head no sparse pattern fits. */
+ * key j <= i: the class the offline profiler assigns to the few heads no
+ * sparse pattern fits (guide, "Phase 1: The Offline Pattern Profiler" and
+ * "Phase 2: The Online Dynamic Kernel Router"), and the prefill MInference is
+ * measured against (guide, "Prefill Latency Benchmark"). */
 enum { MI_PATTERN_ASHAPE = 0, MI_PATTERN_VS = 1, MI_PATTERN_BS = 2, MI_PATTERN_DENSE = 3 };
 
 enum {
@@ -225,6 +227,25 @@ int mi_prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int H
                      int N, int d, float scale, const int8_t* pattern, const mi_params* p,
                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
                      void* stream, void* const* stage_events);
+
+/*
+ * mi_prefill_layer with one mi_params per head: `params` is a HOST array of
+ * Hq entries, read for each head according to its pattern (the pages' offline
+ * pattern profiler sets them per head; guide, "Phase 1: The Offline Pattern
+ * Profiler").  Vertical-Slash
+ * heads may differ in vertical_size and slash_size but must share last_q;
+ * Block-Sparse heads may differ in topk_blocks; A-shape heads in sink and
+ * window.  MI_ERR_INVALID_ARG for VS heads with different last_q.  The
+ * workspace is mi_prefill_workspace_bytes_heads() of the same arguments
+ * (0 if they are invalid).  Everything else as for mi_prefill_layer.
+ */
+size_t mi_prefill_workspace_bytes_heads(int Hq, int Hkv, int N, int d, const int8_t* pattern,
+                                        const mi_params* params);
+int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq,
+                           int Hkv, int N, int d, float scale, const int8_t* pattern,
+                           const mi_params* params, mi_bf16* out, float* lse,
+                           int32_t* err_count, void* ws, size_t ws_bytes, void* stream,
+                           void* const* stage_events);
 
 /*
  * mi_vs_index without a workspace argument.  The paper has no counterpart:

@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = header_functions()
-    assert len(names) == 14
+    assert len(names) == 16
     assert sorted(B.EXPORTS) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -120,6 +120,34 @@ def test_prefill_layer_validation(lib):
     assert lib.mi_prefill_layer(f, f, f, 4, 2, 512, 128, 0.0, good.ctypes.data_as(ctypes.c_void_p),
                                 ctypes.byref(p2), f, None, None, f, 1 << 30, None,
                                 None) == B.MI_ERR_UNSUPPORTED
+
+
+def test_prefill_layer_heads_validation(lib):
+    f = FAKE
+    pat = np.array([1, 1, 2, 0], np.int8)
+    ps = [B.make_params(vertical_size=10 * (h + 1), topk_blocks=h + 1, sink=h, window=h + 8)
+          for h in range(4)]
+    assert B.mi_prefill_workspace_bytes_heads(4, 2, 512, 128, pat, ps) > 0
+    arr = (B.mi_params * 4)(*ps)
+    ok = lib.mi_prefill_layer_heads(f, f, f, 4, 2, 512, 128, 0.0,
+                                    pat.ctypes.data_as(ctypes.c_void_p),
+                                    ctypes.cast(arr, ctypes.c_void_p), f, None, None, f, 16, None,
+                                    None)
+    assert ok == B.MI_ERR_WORKSPACE                      # valid plan, workspace too small
+    ps[1] = B.make_params(last_q=128)                    # VS heads must share last_q
+    arr = (B.mi_params * 4)(*ps)
+    assert lib.mi_prefill_layer_heads(f, f, f, 4, 2, 512, 128, 0.0,
+                                      pat.ctypes.data_as(ctypes.c_void_p),
+                                      ctypes.cast(arr, ctypes.c_void_p), f, None, None, f,
+                                      1 << 30, None, None) == B.MI_ERR_INVALID_ARG
+    assert B.mi_prefill_workspace_bytes_heads(4, 2, 512, 128, pat, ps) == 0
+    ps[1] = B.make_params()
+    ps[3] = B.make_params(window=0)                      # A-shape window >= 1
+    arr = (B.mi_params * 4)(*ps)
+    assert lib.mi_prefill_layer_heads(f, f, f, 4, 2, 512, 128, 0.0,
+                                      pat.ctypes.data_as(ctypes.c_void_p),
+                                      ctypes.cast(arr, ctypes.c_void_p), f, None, None, f,
+                                      1 << 30, None, None) == B.MI_ERR_INVALID_ARG
 
 
 def test_workspace_queries(lib):

@@ -259,6 +259,38 @@ def test_prefill_layer_mixed_matches_oracle(N, d):
         check_attn(out[h], lse[h], ro, rl, what=f"layer h{h} pattern {pattern[h]}")
 
 
+def test_prefill_layer_per_head_parameters():
+    """mi_prefill_layer_heads: every head with its own budgets (VS vertical /
+    slash sizes, BS block count, A-shape sink and window), one launch."""
+    w = synth.workload("mixed_n256k_llama3_8b", Hq=8, Hkv=2, N=1024, d=128)
+    x = synth.make_inputs(w, device="cuda")
+    pattern = np.array([1, 1, 2, 2, 0, 0, 3, 1], np.int8)
+    ps = [B.make_params(vertical_size=20, slash_size=30),
+          B.make_params(vertical_size=60, slash_size=90),
+          B.make_params(topk_blocks=3),
+          B.make_params(topk_blocks=6),
+          B.make_params(sink=64, window=256),
+          B.make_params(sink=10, window=100),
+          B.make_params(),
+          B.make_params(vertical_size=35, slash_size=50)]
+    out, lse = B.mi_prefill_layer_heads(x["q"], x["k"], x["v"], pattern, ps, want_lse=True)
+    torch.cuda.synchronize()
+    for h in range(8):
+        qs, ks_, vs_ = head_slices(x["q"], x["k"], x["v"], h)
+        p = ps[h]
+        if pattern[h] == 0:
+            ro, rl = oracle.attn_ashape(qs, ks_, vs_, 0, p.sink, p.window)
+        elif pattern[h] == 1:
+            a, b, _, _ = oracle.vs_index(qs, ks_, 0, p.last_q, p.vertical_size, p.slash_size)
+            ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, a, b)
+        elif pattern[h] == 2:
+            bi, bc = oracle.bs_index(qs, ks_, 0, p.topk_blocks)
+            ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi, bc)
+        else:
+            ro, rl = oracle.attn_dense(qs, ks_, vs_, 0)
+        check_attn(out[h], lse[h], ro, rl, what=f"per-head h{h} pattern {pattern[h]}")
+
+
 def test_prefill_layer_stage_events_and_stream():
     q, k, v = rand_bf16(4, 1, 512, 128, 16)
     s = torch.cuda.Stream()
