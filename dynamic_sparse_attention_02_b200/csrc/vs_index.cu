@@ -84,7 +84,8 @@ struct TileRegs {
     }
 };
 
-// acc[a][b] = sum_t Qs[t][4ty+a] * Ks[t][4tx+b]
+// acc[a][b] = sum_t Qs[t][4ty+a] * Ks[t][4tx+b]; the operands of step t+1 are
+// loaded while step t's FMAs run
 template <int D>
 __device__ __forceinline__ void dot_4x4(const double* Qs, const double* Ks, int ty, int tx,
                                         double (&acc)[4][4]) {
@@ -92,18 +93,27 @@ __device__ __forceinline__ void dot_4x4(const double* Qs, const double* Ks, int 
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-#pragma unroll 4
+    double2 q01 = *reinterpret_cast<const double2*>(Qs + ty * 4);
+    double2 q23 = *reinterpret_cast<const double2*>(Qs + ty * 4 + 2);
+    double2 k01 = *reinterpret_cast<const double2*>(Ks + tx * 4);
+    double2 k23 = *reinterpret_cast<const double2*>(Ks + tx * 4 + 2);
+#pragma unroll 8
     for (int t = 0; t < D; ++t) {
-        const double2 q01 = *reinterpret_cast<const double2*>(Qs + t * 64 + ty * 4);
-        const double2 q23 = *reinterpret_cast<const double2*>(Qs + t * 64 + ty * 4 + 2);
-        const double2 k01 = *reinterpret_cast<const double2*>(Ks + t * 64 + tx * 4);
-        const double2 k23 = *reinterpret_cast<const double2*>(Ks + t * 64 + tx * 4 + 2);
+        const int tn = t + 1 < D ? t + 1 : t;
+        const double2 nq01 = *reinterpret_cast<const double2*>(Qs + tn * 64 + ty * 4);
+        const double2 nq23 = *reinterpret_cast<const double2*>(Qs + tn * 64 + ty * 4 + 2);
+        const double2 nk01 = *reinterpret_cast<const double2*>(Ks + tn * 64 + tx * 4);
+        const double2 nk23 = *reinterpret_cast<const double2*>(Ks + tn * 64 + tx * 4 + 2);
         const double qa[4] = {q01.x, q01.y, q23.x, q23.y};
         const double kb[4] = {k01.x, k01.y, k23.x, k23.y};
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) acc[a][b] = fma(qa[a], kb[b], acc[a][b]);
+        q01 = nq01;
+        q23 = nq23;
+        k01 = nk01;
+        k23 = nk23;
     }
 }
 
