@@ -474,10 +474,15 @@ int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v,
 
 int mi_debug_wait_failure(int32_t* record8) {
     if (!record8) return MI_ERR_INVALID_ARG;
-    int rec[8];
-    const int rc = cuda_status(read_wait_failure(rec));
+    // attention's record first, else the tensor-core VS score passes' (sites >= 11);
+    // reading clears both
+    int rec[8], rec_vs[8];
+    int rc = cuda_status(read_wait_failure(rec));
     if (rc) return rc;
-    for (int i = 0; i < 8; ++i) record8[i] = rec[i];
+    rc = cuda_status(read_vs_wait_failure(rec_vs));
+    if (rc) return rc;
+    const int* use = rec[1] != 0 ? rec : rec_vs;
+    for (int i = 0; i < 8; ++i) record8[i] = use[i];
     return MI_OK;
 }
 

@@ -1094,40 +1094,13 @@ __global__ void __launch_bounds__(1024) vs_prep_kernel(const int32_t* __restrict
     if (threadIdx.x == 0) ws.vcnt[pos] = min(base_out, ws.vcap);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2-D map over [rows][d] bf16, 64-column x box_rows boxes, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
     using L = Layout<D>;
     CUtensorMap tmQ, tmK, tmV;
-    if (!make_map(&tmQ, a.q, (long long)a.Hq * a.N, D, 128) ||
-        !make_map(&tmK, a.k, (long long)a.Hkv * a.N, D, 64) ||
-        !make_map(&tmV, a.v, (long long)a.Hkv * a.N, D, 64))
+    if (!make_tma_map(&tmQ, a.q, (long long)a.Hq * a.N, D, 128) ||
+        !make_tma_map(&tmK, a.k, (long long)a.Hkv * a.N, D, 64) ||
+        !make_tma_map(&tmV, a.v, (long long)a.Hkv * a.N, D, 64))
         return cudaErrorInvalidValue;
     static unsigned int seq = 0;
     AttnParams p;
@@ -1177,6 +1150,33 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over [rows][d] bf16, 64-column x box_rows boxes, 128-byte swizzle
+bool make_tma_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 cudaError_t read_wait_failure(int* out8) {
     int rec[8];

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -75,6 +76,17 @@ cudaError_t launch_vs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N
                             const VsIndexWs& ws, cudaStream_t st,
                             const int32_t* kv_rows = nullptr, const int32_t* ks_rows = nullptr);
 
+// The two score passes on the tensor cores, for L <= 64 (vs_score_tc.cu).
+// Pass 1 writes ws.m_part / ws.l_part for chunks of kVsTcChunk keys (merge
+// them with nchunks = ceil(N / kVsTcChunk)); pass 2 reads ws.mrow / ws.linv
+// and writes every entry of vscore / sscore [n_heads][N].
+constexpr int kVsTcChunk = 2048;
+cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, int Hkv, int N,
+                                int d, double scale, int L, const HeadList& heads,
+                                const VsIndexWs& ws, float* vscore, float* sscore,
+                                cudaStream_t st);
+cudaError_t read_vs_wait_failure(int* out8);
+
 // ----------------------------------------------------------- BS index
 struct BsIndexWs {
     float* qm;  // [n_heads][nB][d]
@@ -126,6 +138,9 @@ struct AttnLaunch {
     int32_t* err_count;
 };
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);
+// 2-D TMA map over a [rows][d] bf16 matrix: boxes of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill past the last row.
+bool make_tma_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows);
 cudaError_t read_wait_failure(int* out8);
 
 // MI_OK, or MI_ERR_CUDA with the error kept for mi_last_cuda_error().

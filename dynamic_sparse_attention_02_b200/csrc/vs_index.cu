@@ -8,16 +8,18 @@
 // score); the top vertical_size columns and top slash_size diagonals are
 // kept.
 //
-// Two passes over the keys of each head, both on CUDA cores in fp64 (the
-// products of bf16 inputs are exact in fp64, so the scores agree with an
-// fp64 evaluation to rounding level and the ranking matches it):
-//   pass 1 (vs_rowstat): per key chunk, per row, the partial max and sum;
+// Two passes over the keys of each head:
+//   pass 1: per key chunk, per row, the partial max and sum;
 //   merge (vs_rowmerge): once per head, the partials into each row's final
 //     max and 1/sum;
-//   pass 2 (vs_colslash): recompute the probabilities
-//     and reduce them into column sums and diagonal sums in a fixed order
-//     (deterministic).  A chunk owns the diagonals whose first key falls in
-//     it and recomputes the L-1 keys past its end to finish them.
+//   pass 2: recompute the probabilities and reduce them into column sums and
+//     diagonal sums in a fixed order (deterministic).  A chunk owns the
+//     diagonals whose first key falls in it and recomputes the L-1 keys past
+//     its end to finish them.
+// For L <= 64 both passes run on the tensor cores (vs_score_tc.cu: exact bf16
+// products with fp32 accumulation, softmax argument and sums in fp64).  For
+// larger L they run here on CUDA cores in fp64 (vs_rowstat, vs_colslash),
+// where the products of bf16 inputs are exact.
 // Then a block-wide radix top-k per head and list (topk.cuh).
 #include <cfloat>
 
@@ -365,18 +367,31 @@ cudaError_t launch_vs_index_d(const bf16* q, const bf16* k, int Hq, int Hkv, int
     const int nrt = (L + 63) / 64;
     const size_t sm1 = rowstat_smem<D>(), sm2 = colslash_smem<D>(L);
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(vs_rowstat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)sm1)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(vs_colslash_kernel<D>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) !=
-        cudaSuccess)
-        return e;
-    vs_rowstat_kernel<D><<<dim3(nchunks, n, nrt), kThreads, sm1, st>>>(
-        q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.m_part, ws.l_part);
-    vs_rowmerge_kernel<<<n, 64, 0, st>>>(ws.m_part, ws.l_part, L, nchunks, ws.mrow, ws.linv);
-    vs_colslash_kernel<D><<<dim3(nchunks, n), kThreads, sm2, st>>>(
-        q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.mrow, ws.linv, vsc, ssc);
+    if (L <= 64) {
+        // products on the tensor cores (vs_score_tc.cu), same merge
+        if ((e = launch_vs_scores_tc(1, q, k, Hq, Hkv, N, D, scale, L, heads, ws, vsc, ssc, st)) !=
+            cudaSuccess)
+            return e;
+        const int ntc = (N + kVsTcChunk - 1) / kVsTcChunk;
+        vs_rowmerge_kernel<<<n, 64, 0, st>>>(ws.m_part, ws.l_part, L, ntc, ws.mrow, ws.linv);
+        if ((e = launch_vs_scores_tc(2, q, k, Hq, Hkv, N, D, scale, L, heads, ws, vsc, ssc, st)) !=
+            cudaSuccess)
+            return e;
+    } else {
+        if ((e = cudaFuncSetAttribute(vs_rowstat_kernel<D>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(vs_colslash_kernel<D>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) !=
+            cudaSuccess)
+            return e;
+        vs_rowstat_kernel<D><<<dim3(nchunks, n, nrt), kThreads, sm1, st>>>(
+            q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.m_part, ws.l_part);
+        vs_rowmerge_kernel<<<n, 64, 0, st>>>(ws.m_part, ws.l_part, L, nchunks, ws.mrow, ws.linv);
+        vs_colslash_kernel<D><<<dim3(nchunks, n), kThreads, sm2, st>>>(
+            q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.mrow, ws.linv, vsc, ssc);
+    }
     RowCounts rv{}, rs{};
     if (kv_rows) {
         rv.n = n;

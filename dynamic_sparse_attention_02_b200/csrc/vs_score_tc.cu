@@ -1,0 +1,565 @@
+// vs_score_tc.cu -- the Vertical-Slash score passes on the tensor cores
+// (last_q <= 64).
+//
+// MInference 1.0 (hotpaper.ai summary, "key idea"; guide "2. The
+// Vertical-Slash Pattern"): the last L queries of a head score every key
+// column and every diagonal through their causal row softmax.  The products
+// q_i . k_j form a dense contraction, so here they run on tcgen05: one M=128
+// tile stacks the last 64 query rows of two query heads that share a KV head
+// (rows 0-63 the first head, 64-127 the second; for L < 64 the first 64-L
+// rows of each half are padding), and every 128-key tile of K gives
+// S = Q K^T in TMEM (exact bf16 products, fp32 accumulation).
+//
+//   pass 1: per row, the online max and sum of exp over a 2048-key chunk
+//           (exponentials in fp32, the running sum in fp64).  The partials go
+//           to the workspace the CUDA-core passes fill and are merged by
+//           vs_rowmerge into each row's max m_i and 1 / l_i.
+//   pass 2: p_ij = exp(s_ij - m_i) / l_i with the exponent argument in fp64
+//           (exp2 of its fp32 part, times a first-order correction for the
+//           rest), staged in shared memory as fp32 and summed in fp64 per
+//           column and per diagonal in a fixed order.  A chunk owns the
+//           columns it holds and the diagonals whose first key it holds, and
+//           reads one more key tile to finish those diagonals.
+//
+// Warp roles (320 threads): warp 0 loads Q and K tiles by TMA, warp 1 issues
+// the MMAs, warps 2-9 are the epilogue.  TMEM lanes are rows: warp w reads
+// lane quadrant w % 4, and warps 2-5 / 6-9 take key columns 0-63 / 64-127 of
+// each tile.  Two 128-column accumulators let the tensor core fill one while
+// the epilogue drains the other.
+#include <cfloat>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace minfer {
+
+namespace {
+
+constexpr int kTcKeys = 128;     // keys per tile (MMA N)
+constexpr int kTcStages = 2;     // K tiles in flight
+constexpr int kTcThreads = 320;
+constexpr int kEpiWarp0 = 2;     // first epilogue warp
+constexpr int kEpiThreads = 256;
+constexpr int kPStride = 129;    // fp32 words per staged row (conflict-free rows and columns)
+constexpr int kDiag = 191;       // diagonals a 64 x 128 tile touches: u = c - r in [-63, 127]
+constexpr uint32_t kTcTmemCols = 256;
+constexpr double kLog2e = 1.4426950408889634;
+constexpr float kLn2f = 0.69314718055994531f;
+
+// Sequence number of the last launch in which a CTA gave up waiting.
+__device__ unsigned int g_vs_abort_seq = 0;
+// First wait that gave up: {launch seq, site, block x, thread, tile, parity, block y, 0}.
+__device__ int g_vs_wait_fail[8];
+
+enum : int {
+    kSiteTcProducer = 11,
+    kSiteTcMmaQ = 12,
+    kSiteTcMmaK = 13,
+    kSiteTcMmaAcc = 14,
+    kSiteTcEpilogue = 15
+};
+
+__device__ void record_vs_wait_failure(unsigned int seq, int site, int tile, int parity) {
+    if (atomicCAS(&g_vs_wait_fail[1], 0, site) == 0) {
+        g_vs_wait_fail[0] = (int)seq;
+        g_vs_wait_fail[2] = (int)blockIdx.x;
+        g_vs_wait_fail[3] = (int)threadIdx.x;
+        g_vs_wait_fail[4] = tile;
+        g_vs_wait_fail[5] = parity;
+        g_vs_wait_fail[6] = (int)blockIdx.y;
+        __threadfence();
+    }
+}
+
+__device__ __forceinline__ void vs_set_abort(volatile int* abort, unsigned int seq) {
+    *abort = 1;
+    atomicExch(&g_vs_abort_seq, seq);
+}
+
+// Two listed query heads of one KV head per tile; slot 1 may be empty (-1).
+struct PairList {
+    int n;
+    int16_t pos[2][MI_MAX_HEADS];
+};
+
+struct TcParams {
+    HeadList heads;
+    PairList pairs;
+    int Hq, Hkv, N, L, nchunks, chunk;
+    double scale;
+    unsigned int seq;
+    double* m_part;  // pass 1 out: [n_heads][L][nchunks]
+    double* l_part;
+    const double* mrow;  // pass 2 in: [n_heads][L]
+    const double* linv;
+    float* vscore;  // pass 2 out: [n_heads][N]
+    float* sscore;
+};
+
+template <int D, int PASS>
+struct TcLayout {
+    static constexpr int kPanels = D / 64;
+    static constexpr int kQPanel = 128 * 128;      // 128 rows x 128 bytes
+    static constexpr int kKPanel = kTcKeys * 128;  // 128 keys x 128 bytes
+    static constexpr int kKStage = kPanels * kKPanel;
+    static constexpr int q_off = 0;
+    static constexpr int k_off = q_off + kPanels * kQPanel;
+    static constexpr int p_off = k_off + kTcStages * kKStage;
+    static constexpr int p_bytes = PASS == 2 ? 128 * kPStride * 4 : 0;
+    static constexpr int carry_off = p_off + p_bytes;  // [tile parity][slot][64] fp64
+    static constexpr int red_off = carry_off + 2 * 2 * 64 * 8;  // [half][128] x (m, l) fp64
+    static constexpr int bar_off = red_off + 2 * 128 * 2 * 8;
+    static constexpr int kBars = 1 + 2 * kTcStages + 4 + 1;
+    static constexpr int misc_off = bar_off + kBars * 8;
+    static constexpr int bytes = misc_off + 16 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+struct TcBars {
+    uint64_t* q_full;
+    uint64_t* k_full;  // [kTcStages]
+    uint64_t* k_empty;
+    uint64_t* acc_full;  // [2]
+    uint64_t* acc_empty;
+    uint64_t* drain;
+};
+
+// Warp 0, lane 0: Q of both slots once, then the K tiles [jb, jb + 128 t).
+template <int D>
+__device__ void tc_producer(const TcParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                            uint8_t* sm, const TcBars& bars, volatile int* abort, int g, int jb,
+                            int ntiles, int pos_a, int pos_b) {
+    using Lay = TcLayout<D, 1>;
+    prefetch_tmap(tmQ);
+    prefetch_tmap(tmK);
+    const int nslots = pos_b >= 0 ? 2 : 1;
+    mbar_arrive_expect_tx(bars.q_full, (uint32_t)(nslots * Lay::kPanels * 64 * 128));
+    for (int s = 0; s < nslots; ++s) {
+        const int qh = head_qh(p.heads.e[s ? pos_b : pos_a]);
+        const int row = qh * p.N + p.N - 64;
+        for (int pn = 0; pn < Lay::kPanels; ++pn)
+            tma_load_2d(sm + Lay::q_off + pn * Lay::kQPanel + s * 64 * 128, tmQ, 64 * pn, row,
+                        bars.q_full);
+    }
+    int issued = 0;
+    for (int t = 0; t < ntiles; ++t) {
+        const int st = t % kTcStages;
+        if (t >= kTcStages) {
+            const uint32_t par = ((t / kTcStages) - 1) & 1;
+            if (!mbar_wait(&bars.k_empty[st], par, abort)) {
+                if (!*abort) record_vs_wait_failure(p.seq, kSiteTcProducer, t, (int)par);
+                vs_set_abort(abort, p.seq);
+                break;
+            }
+        }
+        mbar_arrive_expect_tx(&bars.k_full[st], (uint32_t)Lay::kKStage);
+        for (int pn = 0; pn < Lay::kPanels; ++pn)
+            tma_load_2d(sm + Lay::k_off + st * Lay::kKStage + pn * Lay::kKPanel, tmK, 64 * pn,
+                        g * p.N + jb + t * kTcKeys, &bars.k_full[st]);
+        issued = t + 1;
+    }
+    // no copy may still be in flight when the CTA exits
+    mbar_wait_budget(bars.q_full, 0);
+    for (int t = issued > kTcStages ? issued - kTcStages : 0; t < issued; ++t)
+        mbar_wait_budget(&bars.k_full[t % kTcStages], (t / kTcStages) & 1);
+}
+
+// Warp 1: per tile, S[buffer t % 2] = Q K_t^T (D / 16 MMAs of 128 x 128 x 16).
+template <int D>
+__device__ void tc_mma(const TcParams& p, uint8_t* sm, const TcBars& bars, volatile int* abort,
+                       uint32_t tmem, int ntiles) {
+    using Lay = TcLayout<D, 1>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t idesc = idesc_bf16_f32(128, kTcKeys, false);
+    tmem = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint32_t q_addr = __shfl_sync(0xffffffffu, smem_u32(sm + Lay::q_off), 0);
+    const uint32_t k_addr = __shfl_sync(0xffffffffu, smem_u32(sm + Lay::k_off), 0);
+    bool ok;
+    {
+        bool w = true;
+        if (lane == 0) {
+            w = mbar_wait(bars.q_full, 0, abort);
+            if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaQ, 0, 0);
+        }
+        ok = __shfl_sync(0xffffffffu, w, 0);
+    }
+    for (int t = 0; ok && t < ntiles; ++t) {
+        const int st = t % kTcStages, b = t & 1;
+        bool w = true;
+        if (lane == 0) {
+            const uint32_t kpar = (t / kTcStages) & 1;
+            w = mbar_wait(&bars.k_full[st], kpar, abort);
+            if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaK, t, (int)kpar);
+            if (w && t >= 2) {
+                const uint32_t apar = ((t >> 1) - 1) & 1;
+                w = mbar_wait(&bars.acc_empty[b], apar, abort);
+                if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaAcc, t, (int)apar);
+            }
+        }
+        ok = __shfl_sync(0xffffffffu, w, 0);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int pn = kk >> 2, off = (kk & 3) * 32;
+            const uint64_t adesc = sw128_desc(q_addr + pn * Lay::kQPanel + off, 16, 1024);
+            const uint64_t bdesc =
+                sw128_desc(k_addr + st * Lay::kKStage + pn * Lay::kKPanel + off, 16, 1024);
+            mma_ss_warp(tmem + 128 * b, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_warp(&bars.acc_full[b]);
+        mma_commit_warp(&bars.k_empty[st]);
+    }
+    if (!ok && lane == 0) vs_set_abort(abort, p.seq);
+    // every MMA must have finished before TMEM is released
+    mma_commit_warp(bars.drain);
+    if (lane == 0) mbar_wait_budget(bars.drain, 0);
+    __syncwarp();
+}
+
+// Epilogue warp: wait for accumulator b of tile t.  A wait that gives up
+// marks the warp failed; a failed warp keeps taking the epilogue's named
+// barriers (so that no other warp waits on it) but touches no data.
+__device__ __forceinline__ bool epi_wait(const TcParams& p, const TcBars& bars,
+                                         volatile int* abort, int t) {
+    const int lane = threadIdx.x & 31;
+    bool w = true;
+    if (lane == 0) {
+        const uint32_t par = (t >> 1) & 1;
+        w = mbar_wait(&bars.acc_full[t & 1], par, abort);
+        if (!w) {
+            if (!*abort) record_vs_wait_failure(p.seq, kSiteTcEpilogue, t, (int)par);
+            vs_set_abort(abort, p.seq);
+        }
+    }
+    return __shfl_sync(0xffffffffu, w, 0);
+}
+
+__device__ __forceinline__ void epi_release(const TcBars& bars, int t) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.acc_empty[t & 1]);
+}
+
+// Keys of a 32-column run starting at key jj that row i takes (j <= i).
+__device__ __forceinline__ int run_valid(bool valid_row, long long i, long long jj) {
+    if (!valid_row) return 0;
+    const long long n = i - jj + 1;
+    return n <= 0 ? 0 : (n >= 32 ? 32 : (int)n);
+}
+
+template <int D, int PASS>
+__device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
+                            volatile int* abort, uint32_t tmem, int jb, int je, int ntiles,
+                            int pos_a, int pos_b, int chunk) {
+    using Lay = TcLayout<D, PASS>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
+    const int quad = warp & 3, half = (warp - kEpiWarp0) >> 2;
+    const int row = 32 * quad + lane;  // tile row = TMEM lane
+    const int slot = row >> 6, r = row & 63;
+    const int pos = slot ? pos_b : pos_a;
+    const int L = p.L, N = p.N, rmin = 64 - L;
+    const bool valid_row = pos >= 0 && r >= rmin;
+    const long long i = (long long)N - 64 + r;  // this row's query position
+    const int rr = r - rmin;                     // its index among the L rows
+    const uint32_t t_row = tmem + ((uint32_t)(32 * quad) << 16) + 64 * half;
+    bool failed = false;
+
+    if (PASS == 1) {
+        // online max (raw dot-product units) and sum of 2^((s - max) * c)
+        const float c = (float)(p.scale * kLog2e);
+        float mraw = -FLT_MAX;
+        double lsum = 0.0;
+        for (int t = 0; t < ntiles; ++t) {
+            if (!failed) failed = !epi_wait(p, bars, abort, t);
+            if (failed) continue;
+            tc_fence_after();
+            const long long j0 = (long long)jb + (long long)t * kTcKeys + 64 * half;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[32];
+                tmem_ld32(t_row + 128 * (t & 1) + 32 * h, v);
+                const int nv = run_valid(valid_row, i, j0 + 32 * h);
+                if (nv > 0) {
+                    float tmax = -FLT_MAX;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        if (u < nv) tmax = fmaxf(tmax, __uint_as_float(v[u]));
+                    if (tmax > mraw) {
+                        if (mraw != -FLT_MAX) lsum *= (double)ex2_approx((mraw - tmax) * c);
+                        mraw = tmax;
+                    }
+                    const float mc = mraw * c;
+                    float s = 0.f;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        if (u < nv) s += ex2_approx(fmaf(__uint_as_float(v[u]), c, -mc));
+                    lsum += (double)s;
+                }
+            }
+            epi_release(bars, t);
+        }
+        // merge the two column halves of each row, then one partial per (row, chunk)
+        double* red = reinterpret_cast<double*>(sm + Lay::red_off);  // [half][128] x (m, l)
+        red[(half * 128 + row) * 2] = mraw == -FLT_MAX ? -DBL_MAX : (double)mraw;
+        red[(half * 128 + row) * 2 + 1] = lsum;
+        epi_bar();
+        if (half == 0 && valid_row && !failed && !*abort) {
+            const double c64 = (double)c;
+            double m = red[row * 2], l = red[row * 2 + 1];
+            const double m1 = red[(128 + row) * 2], l1 = red[(128 + row) * 2 + 1];
+            if (!(m1 == -DBL_MAX || l1 == 0.0)) {
+                if (m == -DBL_MAX || l == 0.0) {
+                    m = m1;
+                    l = l1;
+                } else {
+                    const double mn = fmax(m, m1);
+                    l = l * exp2((m - mn) * c64) + l1 * exp2((m1 - mn) * c64);
+                    m = mn;
+                }
+            }
+            const size_t o = ((size_t)pos * L + rr) * p.nchunks + chunk;
+            p.m_part[o] = l > 0.0 ? m * p.scale : -DBL_MAX;
+            p.l_part[o] = l;
+        }
+        return;
+    }
+
+    // PASS 2
+    float* P = reinterpret_cast<float*>(sm + Lay::p_off);           // [128][kPStride]
+    double* carry = reinterpret_cast<double*>(sm + Lay::carry_off);  // [tile parity][slot][64]
+    double mi = 0.0;
+    float li = 0.f;
+    if (valid_row) {
+        mi = p.mrow[(size_t)pos * L + rr];
+        li = (float)p.linv[(size_t)pos * L + rr];
+    }
+    for (int t = 0; t < ntiles; ++t) {
+        const long long j0 = (long long)jb + (long long)t * kTcKeys;
+        if (!failed) failed = !epi_wait(p, bars, abort, t);
+        if (!failed) {
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[32];
+                tmem_ld32(t_row + 128 * (t & 1) + 32 * h, v);
+                const int c0 = 64 * half + 32 * h;
+                const int nv = run_valid(valid_row, i, j0 + c0);
+                float* prow = P + row * kPStride + c0;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    float pv = 0.f;
+                    if (u < nv) {
+                        // log2 of exp(s * scale - m_i), split into an fp32 part and the rest
+                        const double x =
+                            fma((double)__uint_as_float(v[u]), p.scale, -mi) * kLog2e;
+                        const float x32 = (float)x;
+                        const float lo = (float)(x - (double)x32);
+                        pv = ex2_approx(x32) * fmaf(lo, kLn2f, 1.0f) * li;
+                    }
+                    prow[u] = pv;
+                }
+            }
+            epi_release(bars, t);
+        }
+        epi_bar();  // the tile's probabilities are staged
+        if (!failed && !*abort) {
+            // column sums: thread -> (slot, column)
+            const int cs = et >> 7, cc = et & 127;
+            const int cpos = cs ? pos_b : pos_a;
+            const long long j = j0 + cc;
+            if (cpos >= 0 && j >= jb && j < je) {
+                const float* col = P + (64 * cs) * kPStride + cc;
+                double s = 0.0;
+#pragma unroll 8
+                for (int q = 0; q < 64; ++q) s += (double)col[q * kPStride];
+                p.vscore[(size_t)cpos * N + j] = (float)s;
+            }
+            // diagonal sums: u = c - r; a diagonal that runs past the tile's last
+            // key (u >= 65) is carried into the next tile
+            const int tb = t & 1;
+            for (int dd = et; dd < 2 * kDiag; dd += kEpiThreads) {
+                const int ds = dd >= kDiag ? 1 : 0;
+                const int u = dd - ds * kDiag - 63;
+                const int dpos = ds ? pos_b : pos_a;
+                if (dpos < 0) continue;
+                const int rlo = u < 0 ? -u : 0, rhi = u > 64 ? 127 - u : 63;
+                const float* base = P + (64 * ds) * kPStride + u;
+                double s = 0.0;
+                for (int q = rlo; q <= rhi; ++q) s += (double)base[q * (kPStride + 1)];
+                if (u < 0 && t > 0) s += carry[((tb ^ 1) * 2 + ds) * 64 + (u + 63)];
+                if (u >= 65) {
+                    carry[(tb * 2 + ds) * 64 + (u - 65)] = s;
+                    continue;
+                }
+                const long long o = (long long)N - 64 - j0 - u;
+                if (o < 0 || o >= N) continue;
+                const long long fk = max(0LL, j0 + u + rmin);  // the diagonal's first key
+                if (fk >= jb && fk < je) p.sscore[(size_t)dpos * N + o] = (float)s;
+            }
+        }
+        epi_bar();  // the staging buffer is free again
+    }
+}
+
+template <int D, int PASS>
+__global__ void __launch_bounds__(kTcThreads, PASS == 1 ? 2 : 1)
+    vs_score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ TcParams p) {
+    using Lay = TcLayout<D, PASS>;
+    extern __shared__ uint8_t smem_raw[];
+    // 128-byte swizzled operands need a 1024-byte aligned base
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::bar_off);
+    TcBars bars;
+    bars.q_full = bar;
+    bars.k_full = bar + 1;
+    bars.k_empty = bar + 1 + kTcStages;
+    bars.acc_full = bar + 1 + 2 * kTcStages;
+    bars.acc_empty = bar + 3 + 2 * kTcStages;
+    bars.drain = bar + 5 + 2 * kTcStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::misc_off);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + Lay::misc_off + 4);
+
+    const int pair = blockIdx.x, chunk = blockIdx.y;
+    const int pos_a = p.pairs.pos[0][pair], pos_b = p.pairs.pos[1][pair];
+    const int g = kv_head_of(head_qh(p.heads.e[pos_a]), p.Hq, p.Hkv);
+    const int jb = chunk * p.chunk;
+    const int je = min(p.N, jb + p.chunk);
+    const int jend = PASS == 1 ? je : min(p.N, je + kTcKeys);
+    const int ntiles = (jend - jb + kTcKeys - 1) / kTcKeys;
+    const int warp = threadIdx.x >> 5;
+
+    if (threadIdx.x == 0) {
+        // one read for the whole CTA: every thread must take the same branch
+        *abort = *reinterpret_cast<volatile unsigned int*>(&g_vs_abort_seq) == p.seq ? 1 : 0;
+        mbar_init(bars.q_full, 1);
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&bars.k_full[s], 1);
+            mbar_init(&bars.k_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.acc_full[b], 1);
+            mbar_init(&bars.acc_empty[b], kEpiThreads / 32);
+        }
+        mbar_init(bars.drain, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (*abort) return;  // an earlier CTA of this launch gave up: skip the work
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTcTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if ((threadIdx.x & 31) == 0)
+            tc_producer<D>(p, &tmQ, &tmK, sm, bars, abort, g, jb, ntiles, pos_a, pos_b);
+    } else if (warp == 1) {
+        tc_mma<D>(p, sm, bars, abort, tmem, ntiles);
+        tc_fence_before();
+    } else {
+        tc_epilogue<D, PASS>(p, sm, bars, abort, tmem, jb, je, ntiles, pos_a, pos_b, chunk);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcTmemCols);
+    }
+}
+
+template <int D, int PASS>
+cudaError_t launch_pass(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcParams& p,
+                        cudaStream_t st) {
+    const int smem = TcLayout<D, PASS>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(vs_score_tc_kernel<D, PASS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    vs_score_tc_kernel<D, PASS><<<dim3(p.pairs.n, p.nchunks), kTcThreads, smem, st>>>(tmQ, tmK, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, int Hkv, int N,
+                                int d, double scale, int L, const HeadList& heads,
+                                const VsIndexWs& ws, float* vscore, float* sscore,
+                                cudaStream_t st) {
+    if (heads.n == 0) return cudaSuccess;
+    if (L < 1 || L > 64 || N < 64 || (d != 64 && d != 128)) return cudaErrorInvalidValue;
+    CUtensorMap tmQ, tmK;
+    if (!make_tma_map(&tmQ, q, (long long)Hq * N, d, 64) ||
+        !make_tma_map(&tmK, k, (long long)Hkv * N, d, kTcKeys))
+        return cudaErrorInvalidValue;
+    static unsigned int seq = 0;
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    if (++seq == 0) ++seq;
+    p.seq = seq;
+    p.heads = heads;
+    // pair the listed heads of each KV head in list order; an odd one out runs alone
+    int np = 0;
+    for (int g = 0; g < Hkv; ++g) {
+        int pend = -1;
+        for (int i = 0; i < heads.n; ++i) {
+            if (kv_head_of(head_qh(heads.e[i]), Hq, Hkv) != g) continue;
+            if (pend < 0) {
+                pend = i;
+            } else {
+                p.pairs.pos[0][np] = (int16_t)pend;
+                p.pairs.pos[1][np] = (int16_t)i;
+                ++np;
+                pend = -1;
+            }
+        }
+        if (pend >= 0) {
+            p.pairs.pos[0][np] = (int16_t)pend;
+            p.pairs.pos[1][np] = -1;
+            ++np;
+        }
+    }
+    p.pairs.n = np;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.L = L;
+    p.chunk = kVsTcChunk;
+    p.nchunks = (N + kVsTcChunk - 1) / kVsTcChunk;
+    p.scale = scale;
+    p.m_part = ws.m_part;
+    p.l_part = ws.l_part;
+    p.mrow = ws.mrow;
+    p.linv = ws.linv;
+    p.vscore = vscore;
+    p.sscore = sscore;
+    if (pass == 1)
+        return d == 128 ? launch_pass<128, 1>(tmQ, tmK, p, st) : launch_pass<64, 1>(tmQ, tmK, p, st);
+    return d == 128 ? launch_pass<128, 2>(tmQ, tmK, p, st) : launch_pass<64, 2>(tmQ, tmK, p, st);
+}
+
+cudaError_t read_vs_wait_failure(int* out8) {
+    int rec[8];
+    cudaError_t e = cudaMemcpyFromSymbol(rec, g_vs_wait_fail, sizeof(rec));
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < 8; ++i) out8[i] = rec[i];
+    const int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    return cudaMemcpyToSymbol(g_vs_wait_fail, zero, sizeof(zero));
+}
+
+}  // namespace minfer

@@ -133,7 +133,11 @@ size_t mi_prefill_workspace_bytes(int Hq, int Hkv, int N, int d, const int8_t* p
  * Pattern").  For each listed head h and each of the last L = last_q rows
  * i = N-L .. N-1: row softmax of scale * q_i . k_j over j <= i; vertical[j]
  * sums the probabilities of column j over the L rows, slash[o] sums those of
- * diagonal o = i - j.  Scores are computed in fp64 and ranked as fp32.
+ * diagonal o = i - j.  For last_q <= 64 the products q_i . k_j run on the
+ * tensor cores (exact bf16 products, fp32 accumulation; the softmax argument
+ * and the sums in fp64, the exponentials as fp32 exp2 with an fp64
+ * correction); for larger last_q everything is fp64 on CUDA cores.  Scores
+ * are ranked as fp32.
  * The top vertical_size columns and top slash_size diagonals (ties: lower
  * index first) are written sorted ascending:
  *   v_idx [n_heads][vertical_size], s_idx [n_heads][slash_size] (int32,
@@ -275,12 +279,17 @@ int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int 
 
 /*
  * Diagnostics (not on the hot path; synchronous).  The sparse-attention
- * kernel bounds every wait; the first wait that gives up is recorded as
- * {launch sequence, site, block, thread, group, parity, 0, 0} with site in
- * 1..7 (1 producer/stage-free, 2 MMA/Q, 3 MMA/stage-full, 4 MMA/P-ready,
- * 5 softmax/stage-full, 6 softmax/S-ready, 7 softmax/O-done); site 0 means
- * no wait gave up.  Reading the record copies it to `record8` (host int32
- * [8]) and clears it.  A correct run never records anything.
+ * kernel and the tensor-core Vertical-Slash score passes bound every wait;
+ * the first wait that gives up is recorded as
+ * {launch sequence, site, block, thread, group or tile, parity, 0 or block y,
+ * 0} with site in 1..7 for attention (1 producer/stage-free, 2 MMA/Q,
+ * 3 MMA/stage-full, 4 MMA/P-ready, 5 softmax/stage-full, 6 softmax/S-ready,
+ * 7 softmax/O-done) and 11..15 for the score passes (11 producer/stage-free,
+ * 12 MMA/Q, 13 MMA/stage-full, 14 MMA/accumulator-free, 15 epilogue/
+ * accumulator-full); site 0 means no wait gave up.  Attention's record is
+ * returned when it holds one, else the score passes'.  Reading copies the
+ * record to `record8` (host int32 [8]) and clears both.  A correct run never
+ * records anything.
  */
 int mi_debug_wait_failure(int32_t* record8);
 
