@@ -69,10 +69,32 @@ __device__ void block_radix_select(const Get& get, int n, int k, TopkSmem& s, ui
         for (int b = threadIdx.x; b < 256; b += blockDim.x) s.hist[b] = 0;
         __syncthreads();
         const uint32_t prefix = s.prefix;
-        for (int j = threadIdx.x; j < n; j += blockDim.x) {
-            const uint32_t key = get(j);
-            if ((key & mask) == prefix) atomicAdd(&s.hist[(key >> shift) & 255u], 1u);
+        // a thread's keys mostly share the leading digits (scores of one list
+        // span few binades), so runs of one bin are counted in a register and
+        // added once instead of contending on one shared counter
+        uint32_t run_bin = 0, run_cnt = 0;
+        auto count = [&](uint32_t key) {
+            if ((key & mask) == prefix) {
+                const uint32_t b = (key >> shift) & 255u;
+                if (run_cnt != 0 && b != run_bin) {
+                    atomicAdd(&s.hist[run_bin], run_cnt);
+                    run_cnt = 0;
+                }
+                run_bin = b;
+                ++run_cnt;
+            }
+        };
+        const int bd = (int)blockDim.x;
+        int j = threadIdx.x;
+        for (; j + 7 * bd < n; j += 8 * bd) {  // eight loads in flight per thread
+            uint32_t kb[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kb[u] = get(j + u * bd);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) count(kb[u]);
         }
+        for (; j < n; j += bd) count(get(j));
+        if (run_cnt != 0) atomicAdd(&s.hist[run_bin], run_cnt);
         __syncthreads();
         if (threadIdx.x == 0) {
             int rem = s.remaining;
@@ -93,26 +115,85 @@ __device__ void block_radix_select(const Get& get, int n, int k, TopkSmem& s, ui
     __syncthreads();
 }
 
-// Write the selected indices in ascending order to out[0..k).
+// Write the selected indices in ascending order to out[0..k): every key > thr
+// and the first need_eq keys == thr.  Each warp owns one contiguous segment of
+// the keys and reads it 32 keys at a time (coalesced); one scan over the warps
+// (equal keys before the segment, selections before it) places its output,
+// and ballots order the lanes within each 32-key step.
+struct CompactSmem {
+    int eq[32], sel[32];
+};
 template <class Get>
 __device__ void block_select_compact(const Get& get, int n, int k, uint32_t thr, int need_eq,
                                      TopkSmem& s, int32_t* out) {
-    int eq_base = 0, sel_base = 0;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int j = base + threadIdx.x;
-        uint32_t key = 0;
-        if (j < n) key = get(j);
-        const int gt = (j < n && key > thr) ? 1 : 0;
-        const int eq = (j < n && key == thr) ? 1 : 0;
-        int eq_tot;
-        const int eq_rank = eq_base + block_exclusive_scan(eq, s.warp_tot, eq_tot);
-        const int sel = gt | (eq & (eq_rank < need_eq ? 1 : 0));
-        int sel_tot;
-        const int pos = sel_base + block_exclusive_scan(sel, s.warp_tot, sel_tot);
-        if (sel && pos < k) out[pos] = j;
-        eq_base += eq_tot;
-        sel_base += sel_tot;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const int per = (((n + nw - 1) / nw) + 31) & ~31;
+    const int j0 = min(n, w * per), j1 = min(n, j0 + per);
+    int gt = 0, eq = 0;
+    for (int base = j0; base < j1; base += 128) {
+        uint32_t kb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = base + 32 * u + lane;
+            kb[u] = j < j1 ? get(j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool in = base + 32 * u + lane < j1;
+            gt += (in && kb[u] > thr) ? 1 : 0;
+            eq += (in && kb[u] == thr) ? 1 : 0;
+        }
     }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    CompactSmem* cs = reinterpret_cast<CompactSmem*>(s.hist);  // the histogram is done
+    __syncthreads();
+    if (lane == 0) {
+        cs->eq[w] = eq;
+        cs->sel[w] = gt;
+    }
+    __syncthreads();
+    if (w == 0) {
+        const int e = lane < nw ? cs->eq[lane] : 0, g = lane < nw ? cs->sel[lane] : 0;
+        int ei = e;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ei, off);
+            if (lane >= off) ei += y;
+        }
+        const int e_before = ei - e;
+        const int take = max(0, min(e, need_eq - e_before));
+        const int sv = g + take;
+        int si = sv;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, si, off);
+            if (lane >= off) si += y;
+        }
+        __syncwarp();
+        if (lane < nw) {
+            cs->eq[lane] = e_before;
+            cs->sel[lane] = si - sv;
+        }
+    }
+    __syncthreads();
+    int eq_seen = cs->eq[w], pos = cs->sel[w];
+    const int end = pos + gt + max(0, min(eq, need_eq - eq_seen));
+    for (int base = j0; base < j1 && pos < end; base += 32) {
+        const int j = base + lane;
+        const uint32_t key = j < j1 ? get(j) : 0u;
+        const bool g1 = j < j1 && key > thr;
+        const bool e1 = j < j1 && key == thr;
+        const unsigned eqm = __ballot_sync(0xffffffffu, e1);
+        const bool sel = g1 || (e1 && eq_seen + __popc(eqm & below) < need_eq);
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        const int p = pos + __popc(selm & below);
+        if (sel && p < k) out[p] = j;
+        eq_seen += __popc(eqm);
+        pos += __popc(selm);
+    }
+    __syncthreads();
 }
 
 // ---- one warp per selection (many short rows at once), same contract as above.

@@ -326,21 +326,32 @@ struct GlobalKeys {
     __device__ uint32_t operator()(int j) const { return float_order_key(p[j]); }
 };
 
-// Top-k of each row of scores [rows][n]; out row stride out_stride, -1 past k.
-__global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict__ scores,
-                                                         int n, int k, int32_t* out,
-                                                         int out_stride, RowCounts rk) {
+// One batched top-k: rows of scores [rows][n], output row stride out_stride,
+// -1 past each row's k.
+struct TopkJob {
+    const float* scores;
+    int32_t* out;
+    int k, out_stride;
+    RowCounts rk;
+};
+
+// Blocks [0, rows) take job a, blocks [rows, 2 rows) job b.
+__global__ void __launch_bounds__(1024) topk_rows_kernel(int n, int rows,
+                                                         const __grid_constant__ TopkJob a,
+                                                         const __grid_constant__ TopkJob b) {
     __shared__ TopkSmem s;
-    const int row = blockIdx.x;
-    int32_t* o = out + (size_t)row * out_stride;
-    const int kk = min(row < rk.n ? rk.k[row] : k, n);
-    for (int t = kk + threadIdx.x; t < out_stride; t += blockDim.x) o[t] = -1;
+    const bool second = (int)blockIdx.x >= rows;
+    const TopkJob* job = second ? &b : &a;
+    const int row = (int)blockIdx.x - (second ? rows : 0);
+    int32_t* o = job->out + (size_t)row * job->out_stride;
+    const int kk = min(row < job->rk.n ? job->rk.k[row] : job->k, n);
+    for (int t = kk + threadIdx.x; t < job->out_stride; t += blockDim.x) o[t] = -1;
     if (kk <= 0) return;
     if (kk == n) {
         for (int j = threadIdx.x; j < n; j += blockDim.x) o[j] = j;
         return;
     }
-    GlobalKeys get{scores + (size_t)row * n};
+    GlobalKeys get{job->scores + (size_t)row * n};
     uint32_t thr;
     int need_eq;
     block_radix_select(get, n, kk, s, thr, need_eq);
@@ -392,17 +403,16 @@ cudaError_t launch_vs_index_d(const bf16* q, const bf16* k, int Hq, int Hkv, int
         vs_colslash_kernel<D><<<dim3(nchunks, n), kThreads, sm2, st>>>(
             q, k, Hq, Hkv, N, L, nchunks, heads, scale, ws.mrow, ws.linv, vsc, ssc);
     }
-    RowCounts rv{}, rs{};
+    TopkJob jv{vsc, v_idx, kv, kv, {}}, js{ssc, s_idx, ks, ks, {}};
     if (kv_rows) {
-        rv.n = n;
-        for (int i = 0; i < n; ++i) rv.k[i] = kv_rows[i];
+        jv.rk.n = n;
+        for (int i = 0; i < n; ++i) jv.rk.k[i] = kv_rows[i];
     }
     if (ks_rows) {
-        rs.n = n;
-        for (int i = 0; i < n; ++i) rs.k[i] = ks_rows[i];
+        js.rk.n = n;
+        for (int i = 0; i < n; ++i) js.rk.k[i] = ks_rows[i];
     }
-    topk_rows_kernel<<<n, 1024, 0, st>>>(vsc, N, kv, v_idx, kv, rv);
-    topk_rows_kernel<<<n, 1024, 0, st>>>(ssc, N, ks, s_idx, ks, rs);
+    topk_rows_kernel<<<2 * n, 1024, 0, st>>>(N, n, jv, js);
     return cudaGetLastError();
 }
 

@@ -14,17 +14,18 @@
 //           (exponentials in fp32, the running sum in fp64).  The partials go
 //           to the workspace the CUDA-core passes fill and are merged by
 //           vs_rowmerge into each row's max m_i and 1 / l_i.
-//   pass 2: p_ij = exp(s_ij - m_i) / l_i with the exponent argument in fp64
-//           (exp2 of its fp32 part, times a first-order correction for the
-//           rest), staged in shared memory as fp32 and summed in fp64 per
-//           column and per diagonal in a fixed order.  A chunk owns the
+//   pass 2: p_ij = exp(s_ij - m_i) / l_i with the exponent carried as an
+//           unevaluated pair of fp32 values (exp2 of the leading part times a
+//           first-order correction for the rest), staged in shared memory as
+//           fp32 and summed per column and per diagonal with compensated
+//           (Kahan) fp32 sums in a fixed order.  A chunk owns the
 //           columns it holds and the diagonals whose first key it holds, and
 //           reads one more key tile to finish those diagonals.
 //
-// Warp roles (320 threads): warp 0 loads Q and K tiles by TMA, warp 1 issues
-// the MMAs, warps 2-9 are the epilogue.  TMEM lanes are rows: warp w reads
-// lane quadrant w % 4, and warps 2-5 / 6-9 take key columns 0-63 / 64-127 of
-// each tile.  Two 128-column accumulators let the tensor core fill one while
+// Warp roles: warp 0 loads Q and K tiles by TMA, warp 1 issues the MMAs,
+// warps 2.. are the epilogue (8 in pass 1, 16 in pass 2).  TMEM lanes are
+// rows: warp w reads lane quadrant w % 4, and the epilogue warps of one
+// quadrant split the tile's 128 key columns between them.  Two 128-column accumulators let the tensor core fill one while
 // the epilogue drains the other.
 #include <cfloat>
 
@@ -37,10 +38,12 @@ namespace {
 
 constexpr int kTcKeys = 128;     // keys per tile (MMA N)
 constexpr int kTcStages = 2;     // K tiles in flight
-constexpr int kTcThreads = 320;
 constexpr int kEpiWarp0 = 2;     // first epilogue warp
-constexpr int kEpiThreads = 256;
-constexpr int kPStride = 129;    // fp32 words per staged row (conflict-free rows and columns)
+// Staged probabilities are skewed: row r of a slot keeps key column c at
+// position c - r + 63, so diagonal u = c - r is position u + 63 of every row.
+// 192 words per row (191 used): row stride 192 - 1 = 191 is odd, so the
+// 32 rows of a warp store one column to 32 distinct banks.
+constexpr int kSkew = 192;
 constexpr int kDiag = 191;       // diagonals a 64 x 128 tile touches: u = c - r in [-63, 127]
 constexpr uint32_t kTcTmemCols = 256;
 constexpr double kLog2e = 1.4426950408889634;
@@ -96,6 +99,18 @@ struct TcParams {
     float* sscore;
 };
 
+// Epilogue width per pass: pass 1 runs two CTAs per SM with 8 epilogue warps
+// (64 key columns each), pass 2 one CTA per SM with 16 (32 columns each), so
+// that each SM sub-partition holds four epilogue warps in both.
+template <int PASS>
+struct TcShape {
+    static constexpr int kEpiWarps = PASS == 1 ? 8 : 16;
+    static constexpr int kEpiThreads = kEpiWarps * 32;
+    static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+    static constexpr int kGroups = kEpiWarps / 4;   // column groups per lane quadrant
+    static constexpr int kCols = kTcKeys / kGroups;  // key columns per epilogue warp
+};
+
 template <int D, int PASS>
 struct TcLayout {
     static constexpr int kPanels = D / 64;
@@ -105,10 +120,10 @@ struct TcLayout {
     static constexpr int q_off = 0;
     static constexpr int k_off = q_off + kPanels * kQPanel;
     static constexpr int p_off = k_off + kTcStages * kKStage;
-    static constexpr int p_bytes = PASS == 2 ? 128 * kPStride * 4 : 0;
+    static constexpr int p_bytes = PASS == 2 ? 2 * 64 * kSkew * 4 : 0;
     static constexpr int carry_off = p_off + p_bytes;  // [tile parity][slot][64] fp64
-    static constexpr int red_off = carry_off + 2 * 2 * 64 * 8;  // [half][128] x (m, l) fp64
-    static constexpr int bar_off = red_off + 2 * 128 * 2 * 8;
+    static constexpr int red_off = carry_off + 2 * 2 * 64 * 8;  // [group][128] x (m, l) fp64
+    static constexpr int bar_off = red_off + TcShape<PASS>::kGroups * 128 * 2 * 8;
     static constexpr int kBars = 1 + 2 * kTcStages + 4 + 1;
     static constexpr int misc_off = bar_off + kBars * 8;
     static constexpr int bytes = misc_off + 16 + 1024;  // + alignment slack
@@ -120,8 +135,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+template <int PASS>
 __device__ __forceinline__ void epi_bar() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(TcShape<PASS>::kEpiThreads) : "memory");
 }
 
 struct TcBars {
@@ -250,6 +266,32 @@ __device__ __forceinline__ void epi_release(const TcBars& bars, int t) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.acc_empty[t & 1]);
 }
 
+// 2^(s c - m') for c = c_hi + c_lo and m' = m_hi + m_lo: the product's rounding
+// error (FMA residual) and the subtraction's (TwoSum) are kept, and 2^x of the
+// small remainder x is taken as 1 + x ln 2 around the MUFU exp2 of the rest.
+__device__ __forceinline__ float prob(float s, float c_hi, float c_lo, float m_hi, float m_lo) {
+    const float p1 = s * c_hi;
+    const float e1 = fmaf(s, c_hi, -p1);  // exact: s * c_hi = p1 + e1
+    const float y = p1 - m_hi;
+    const float bb = y - p1;
+    const float e2 = (p1 - (y - bb)) + (-m_hi - bb);  // exact: p1 - m_hi = y + e2
+    const float lo = e1 + e2 + fmaf(s, c_lo, -m_lo);
+    return ex2_approx(y) * fmaf(lo, kLn2f, 1.0f);
+}
+
+// Compensated fp32 sum of non-negative terms (error about one rounding of the
+// result, whatever the count).
+struct KahanSum {
+    float s = 0.f, c = 0.f;
+    __device__ __forceinline__ void add(float x) {
+        const float y = x - c;
+        const float t = s + y;
+        c = (t - s) - y;
+        s = t;
+    }
+    __device__ __forceinline__ double value() const { return (double)s - (double)c; }
+};
+
 // Keys of a 32-column run starting at key jj that row i takes (j <= i).
 __device__ __forceinline__ int run_valid(bool valid_row, long long i, long long jj) {
     if (!valid_row) return 0;
@@ -262,9 +304,10 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                             volatile int* abort, uint32_t tmem, int jb, int je, int ntiles,
                             int pos_a, int pos_b, int chunk) {
     using Lay = TcLayout<D, PASS>;
+    using Sh = TcShape<PASS>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
-    const int quad = warp & 3, half = (warp - kEpiWarp0) >> 2;
+    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. kEpiThreads - 1
+    const int quad = warp & 3, grp = (warp - kEpiWarp0) >> 2;
     const int row = 32 * quad + lane;  // tile row = TMEM lane
     const int slot = row >> 6, r = row & 63;
     const int pos = slot ? pos_b : pos_a;
@@ -272,7 +315,7 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
     const bool valid_row = pos >= 0 && r >= rmin;
     const long long i = (long long)N - 64 + r;  // this row's query position
     const int rr = r - rmin;                     // its index among the L rows
-    const uint32_t t_row = tmem + ((uint32_t)(32 * quad) << 16) + 64 * half;
+    const uint32_t t_row = tmem + ((uint32_t)(32 * quad) << 16) + Sh::kCols * grp;
     bool failed = false;
 
     if (PASS == 1) {
@@ -284,9 +327,9 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
             if (!failed) failed = !epi_wait(p, bars, abort, t);
             if (failed) continue;
             tc_fence_after();
-            const long long j0 = (long long)jb + (long long)t * kTcKeys + 64 * half;
+            const long long j0 = (long long)jb + (long long)t * kTcKeys + Sh::kCols * grp;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < Sh::kCols / 32; ++h) {
                 uint32_t v[32];
                 tmem_ld32(t_row + 128 * (t & 1) + 32 * h, v);
                 const int nv = run_valid(valid_row, i, j0 + 32 * h);
@@ -310,11 +353,11 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
             epi_release(bars, t);
         }
         // merge the two column halves of each row, then one partial per (row, chunk)
-        double* red = reinterpret_cast<double*>(sm + Lay::red_off);  // [half][128] x (m, l)
-        red[(half * 128 + row) * 2] = mraw == -FLT_MAX ? -DBL_MAX : (double)mraw;
-        red[(half * 128 + row) * 2 + 1] = lsum;
-        epi_bar();
-        if (half == 0 && valid_row && !failed && !*abort) {
+        double* red = reinterpret_cast<double*>(sm + Lay::red_off);  // [group][128] x (m, l)
+        red[(grp * 128 + row) * 2] = mraw == -FLT_MAX ? -DBL_MAX : (double)mraw;
+        red[(grp * 128 + row) * 2 + 1] = lsum;
+        epi_bar<PASS>();
+        if (grp == 0 && valid_row && !failed && !*abort) {
             const double c64 = (double)c;
             double m = red[row * 2], l = red[row * 2 + 1];
             const double m1 = red[(128 + row) * 2], l1 = red[(128 + row) * 2 + 1];
@@ -336,67 +379,81 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
     }
 
     // PASS 2
-    float* P = reinterpret_cast<float*>(sm + Lay::p_off);           // [128][kPStride]
+    float* P = reinterpret_cast<float*>(sm + Lay::p_off);           // [slot][64][kSkew]
     double* carry = reinterpret_cast<double*>(sm + Lay::carry_off);  // [tile parity][slot][64]
-    double mi = 0.0;
-    float li = 0.f;
+    // log2 e * (s * scale - m_i) = s * c - m' with c and m' as unevaluated fp32
+    // pairs (hi + lo), so the exponent keeps ~48 bits without fp64 arithmetic
+    const double c64 = p.scale * kLog2e;
+    const float c_hi = (float)c64, c_lo = (float)(c64 - (double)c_hi);
+    float m_hi = 0.f, m_lo = 0.f, li = 0.f;
     if (valid_row) {
-        mi = p.mrow[(size_t)pos * L + rr];
+        const double mq = p.mrow[(size_t)pos * L + rr] * kLog2e;
+        m_hi = (float)mq;
+        m_lo = (float)(mq - (double)m_hi);
         li = (float)p.linv[(size_t)pos * L + rr];
     }
+    // positions outside a row's 128 keys are never written: zero them once
+    for (int x = et; x < 2 * 64 * kSkew; x += Sh::kEpiThreads) P[x] = 0.f;
+    epi_bar<PASS>();
+    float* const prow_base = P + slot * 64 * kSkew + r * (kSkew - 1) + 63;  // + column c
     for (int t = 0; t < ntiles; ++t) {
         const long long j0 = (long long)jb + (long long)t * kTcKeys;
         if (!failed) failed = !epi_wait(p, bars, abort, t);
         if (!failed) {
             tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < Sh::kCols / 32; ++h) {
                 uint32_t v[32];
                 tmem_ld32(t_row + 128 * (t & 1) + 32 * h, v);
-                const int c0 = 64 * half + 32 * h;
+                const int c0 = Sh::kCols * grp + 32 * h;
                 const int nv = run_valid(valid_row, i, j0 + c0);
-                float* prow = P + row * kPStride + c0;
+                float* prow = prow_base + c0;
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                     float pv = 0.f;
-                    if (u < nv) {
-                        // log2 of exp(s * scale - m_i), split into an fp32 part and the rest
-                        const double x =
-                            fma((double)__uint_as_float(v[u]), p.scale, -mi) * kLog2e;
-                        const float x32 = (float)x;
-                        const float lo = (float)(x - (double)x32);
-                        pv = ex2_approx(x32) * fmaf(lo, kLn2f, 1.0f) * li;
-                    }
+                    if (u < nv) pv = prob(__uint_as_float(v[u]), c_hi, c_lo, m_hi, m_lo) * li;
                     prow[u] = pv;
                 }
             }
             epi_release(bars, t);
         }
-        epi_bar();  // the tile's probabilities are staged
+        epi_bar<PASS>();  // the tile's probabilities are staged
         if (!failed && !*abort) {
-            // column sums: thread -> (slot, column)
-            const int cs = et >> 7, cc = et & 127;
-            const int cpos = cs ? pos_b : pos_a;
-            const long long j = j0 + cc;
-            if (cpos >= 0 && j >= jb && j < je) {
-                const float* col = P + (64 * cs) * kPStride + cc;
-                double s = 0.0;
-#pragma unroll 8
-                for (int q = 0; q < 64; ++q) s += (double)col[q * kPStride];
-                p.vscore[(size_t)cpos * N + j] = (float)s;
-            }
-            // diagonal sums: u = c - r; a diagonal that runs past the tile's last
-            // key (u >= 65) is carried into the next tile
+            // 256 column sums (slot, column) then 2 x 191 diagonal sums (slot,
+            // u = c - r), dealt round-robin over the epilogue threads; a diagonal
+            // that runs past the tile's last key (u >= 65) is carried into the
+            // next tile
             const int tb = t & 1;
-            for (int dd = et; dd < 2 * kDiag; dd += kEpiThreads) {
+            for (int rd = et; rd < 256 + 2 * kDiag; rd += Sh::kEpiThreads) {
+                if (rd < 256) {
+                    const int cs = rd >> 7, cc = rd & 127;
+                    const int cpos = cs ? pos_b : pos_a;
+                    const long long j = j0 + cc;
+                    if (cpos < 0 || j < jb || j >= je) continue;
+                    const float* col = P + cs * 64 * kSkew + cc + 63;  // row q at q * (kSkew - 1)
+                    KahanSum ks[4];  // four independent chains (rows q mod 4)
+#pragma unroll
+                    for (int q = 0; q < 64; q += 4) {
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) ks[w].add(col[(q + w) * (kSkew - 1)]);
+                    }
+                    p.vscore[(size_t)cpos * N + j] =
+                        (float)((ks[0].value() + ks[1].value()) + (ks[2].value() + ks[3].value()));
+                    continue;
+                }
+                const int dd = rd - 256;
                 const int ds = dd >= kDiag ? 1 : 0;
                 const int u = dd - ds * kDiag - 63;
                 const int dpos = ds ? pos_b : pos_a;
                 if (dpos < 0) continue;
-                const int rlo = u < 0 ? -u : 0, rhi = u > 64 ? 127 - u : 63;
-                const float* base = P + (64 * ds) * kPStride + u;
-                double s = 0.0;
-                for (int q = rlo; q <= rhi; ++q) s += (double)base[q * (kPStride + 1)];
+                const float* dcol = P + ds * 64 * kSkew + u + 63;  // row q at q * kSkew
+                KahanSum ks[4];  // four chains; positions past a row's keys hold 0
+#pragma unroll
+                for (int q = 0; q < 64; q += 4) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) ks[w].add(dcol[(q + w) * kSkew]);
+                }
+                double s = (ks[0].value() + ks[1].value()) + (ks[2].value() + ks[3].value());
                 if (u < 0 && t > 0) s += carry[((tb ^ 1) * 2 + ds) * 64 + (u + 63)];
                 if (u >= 65) {
                     carry[(tb * 2 + ds) * 64 + (u - 65)] = s;
@@ -408,12 +465,12 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                 if (fk >= jb && fk < je) p.sscore[(size_t)dpos * N + o] = (float)s;
             }
         }
-        epi_bar();  // the staging buffer is free again
+        epi_bar<PASS>();  // the staging buffer is free again
     }
 }
 
 template <int D, int PASS>
-__global__ void __launch_bounds__(kTcThreads, PASS == 1 ? 2 : 1)
+__global__ void __launch_bounds__(TcShape<PASS>::kThreads, PASS == 1 ? 2 : 1)
     vs_score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ TcParams p) {
@@ -452,7 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, PASS == 1 ? 2 : 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.acc_full[b], 1);
-            mbar_init(&bars.acc_empty[b], kEpiThreads / 32);
+            mbar_init(&bars.acc_empty[b], TcShape<PASS>::kEpiWarps);
         }
         mbar_init(bars.drain, 1);
         fence_mbar_init();
@@ -491,7 +548,8 @@ cudaError_t launch_pass(const CUtensorMap& tmQ, const CUtensorMap& tmK, const Tc
     cudaError_t e = cudaFuncSetAttribute(vs_score_tc_kernel<D, PASS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    vs_score_tc_kernel<D, PASS><<<dim3(p.pairs.n, p.nchunks), kTcThreads, smem, st>>>(tmQ, tmK, p);
+    vs_score_tc_kernel<D, PASS>
+        <<<dim3(p.pairs.n, p.nchunks), TcShape<PASS>::kThreads, smem, st>>>(tmQ, tmK, p);
     return cudaGetLastError();
 }
 
