@@ -266,30 +266,74 @@ __device__ __forceinline__ void epi_release(const TcBars& bars, int t) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.acc_empty[t & 1]);
 }
 
-// 2^(s c - m') for c = c_hi + c_lo and m' = m_hi + m_lo: the product's rounding
-// error (FMA residual) and the subtraction's (TwoSum) are kept, and 2^x of the
-// small remainder x is taken as 1 + x ln 2 around the MUFU exp2 of the rest.
-__device__ __forceinline__ float prob(float s, float c_hi, float c_lo, float m_hi, float m_lo) {
-    const float p1 = s * c_hi;
-    const float e1 = fmaf(s, c_hi, -p1);  // exact: s * c_hi = p1 + e1
-    const float y = p1 - m_hi;
-    const float bb = y - p1;
-    const float e2 = (p1 - (y - bb)) + (-m_hi - bb);  // exact: p1 - m_hi = y + e2
-    const float lo = e1 + e2 + fmaf(s, c_lo, -m_lo);
-    return ex2_approx(y) * fmaf(lo, kLn2f, 1.0f);
+// p = 2^(s c - m') for c = c_hi + c_lo and m' = m_hi + m_lo (prob2 below):
+// the product's rounding error (FMA residual) and the subtraction's (TwoSum)
+// are kept, and 2^x of the small remainder x is taken as 1 + x ln 2 around the
+// MUFU exp2 of the rest.
+// ---- packed pairs of fp32 (sm_100 f32x2 arithmetic: two IEEE round-to-
+// nearest operations per instruction, the same results as two scalar ones)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ void upk2(uint64_t d, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(d));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
-// Compensated fp32 sum of non-negative terms (error about one rounding of the
-// result, whatever the count).
-struct KahanSum {
-    float s = 0.f, c = 0.f;
-    __device__ __forceinline__ void add(float x) {
-        const float y = x - c;
-        const float t = s + y;
-        c = (t - s) - y;
+// prob() for two scores at once; the constants come packed (both halves
+// equal): nchi = -c_hi, chi = c_hi, mhi = m_hi, clo = c_lo, nmlo = -m_lo.
+__device__ __forceinline__ uint64_t prob2(uint64_t s2, uint64_t nchi, uint64_t chi, uint64_t mhi,
+                                          uint64_t clo, uint64_t nmlo, uint64_t ln2,
+                                          uint64_t one) {
+    const uint64_t np1 = mul2(s2, nchi);   // -p1, p1 = fl(s c_hi)
+    const uint64_t e1 = fma2(s2, chi, np1);  // exact: s c_hi = p1 + e1
+    const uint64_t ny = add2(np1, mhi);      // -y, y = fl(p1 - m_hi)
+    const uint64_t bb = sub2(ny, np1);
+    const uint64_t e2 = add2(sub2(np1, sub2(ny, bb)), sub2(mhi, bb));  // exact: -p1 + m_hi = -y + e2
+    const uint64_t lo = add2(add2(e1, e2), fma2(s2, clo, nmlo));       // s c - m' = y + lo
+    float y0, y1;
+    upk2(ny, y0, y1);
+    const uint64_t ex = pk2(ex2_approx(-y0), ex2_approx(-y1));
+    return mul2(ex, fma2(lo, ln2, one));
+}
+
+// Two compensated fp32 sums of non-negative terms side by side (error about
+// one rounding of each result, whatever the count).
+struct KahanSum2 {
+    uint64_t s = 0, c = 0;
+    __device__ __forceinline__ void add(uint64_t x) {
+        const uint64_t y = sub2(x, c);
+        const uint64_t t = add2(s, y);
+        c = sub2(sub2(t, s), y);
         s = t;
     }
-    __device__ __forceinline__ double value() const { return (double)s - (double)c; }
+    __device__ __forceinline__ double value() const {
+        float s0, s1, c0, c1;
+        upk2(s, s0, s1);
+        upk2(c, c0, c1);
+        return ((double)s0 - (double)c0) + ((double)s1 - (double)c1);
+    }
 };
 
 // Keys of a 32-column run starting at key jj that row i takes (j <= i).
@@ -392,6 +436,9 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
         m_lo = (float)(mq - (double)m_hi);
         li = (float)p.linv[(size_t)pos * L + rr];
     }
+    const uint64_t k_nchi = pk2(-c_hi, -c_hi), k_chi = pk2(c_hi, c_hi), k_mhi = pk2(m_hi, m_hi);
+    const uint64_t k_clo = pk2(c_lo, c_lo), k_nmlo = pk2(-m_lo, -m_lo), k_li = pk2(li, li);
+    const uint64_t k_ln2 = pk2(kLn2f, kLn2f), k_one = pk2(1.f, 1.f);
     // positions outside a row's 128 keys are never written: zero them once
     for (int x = et; x < 2 * 64 * kSkew; x += Sh::kEpiThreads) P[x] = 0.f;
     epi_bar<PASS>();
@@ -409,10 +456,15 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                 const int nv = run_valid(valid_row, i, j0 + c0);
                 float* prow = prow_base + c0;
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    float pv = 0.f;
-                    if (u < nv) pv = prob(__uint_as_float(v[u]), c_hi, c_lo, m_hi, m_lo) * li;
-                    prow[u] = pv;
+                for (int u = 0; u < 32; u += 2) {
+                    const uint64_t p2 = mul2(
+                        prob2(pk2(__uint_as_float(v[u]), __uint_as_float(v[u + 1])), k_nchi,
+                              k_chi, k_mhi, k_clo, k_nmlo, k_ln2, k_one),
+                        k_li);
+                    float p0, p1;
+                    upk2(p2, p0, p1);
+                    prow[u] = u < nv ? p0 : 0.f;
+                    prow[u + 1] = u + 1 < nv ? p1 : 0.f;
                 }
             }
             epi_release(bars, t);
@@ -431,14 +483,15 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                     const long long j = j0 + cc;
                     if (cpos < 0 || j < jb || j >= je) continue;
                     const float* col = P + cs * 64 * kSkew + cc + 63;  // row q at q * (kSkew - 1)
-                    KahanSum ks[4];  // four independent chains (rows q mod 4)
+                    KahanSum2 ks[2];  // four independent chains (rows q mod 4) in two pairs
 #pragma unroll
                     for (int q = 0; q < 64; q += 4) {
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) ks[w].add(col[(q + w) * (kSkew - 1)]);
+                        for (int w = 0; w < 2; ++w)
+                            ks[w].add(pk2(col[(q + 2 * w) * (kSkew - 1)],
+                                          col[(q + 2 * w + 1) * (kSkew - 1)]));
                     }
-                    p.vscore[(size_t)cpos * N + j] =
-                        (float)((ks[0].value() + ks[1].value()) + (ks[2].value() + ks[3].value()));
+                    p.vscore[(size_t)cpos * N + j] = (float)(ks[0].value() + ks[1].value());
                     continue;
                 }
                 const int dd = rd - 256;
@@ -447,13 +500,14 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                 const int dpos = ds ? pos_b : pos_a;
                 if (dpos < 0) continue;
                 const float* dcol = P + ds * 64 * kSkew + u + 63;  // row q at q * kSkew
-                KahanSum ks[4];  // four chains; positions past a row's keys hold 0
+                KahanSum2 ks[2];  // four chains in two pairs; positions past a row's keys hold 0
 #pragma unroll
                 for (int q = 0; q < 64; q += 4) {
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) ks[w].add(dcol[(q + w) * kSkew]);
+                    for (int w = 0; w < 2; ++w)
+                        ks[w].add(pk2(dcol[(q + 2 * w) * kSkew], dcol[(q + 2 * w + 1) * kSkew]));
                 }
-                double s = (ks[0].value() + ks[1].value()) + (ks[2].value() + ks[3].value());
+                double s = ks[0].value() + ks[1].value();
                 if (u < 0 && t > 0) s += carry[((tb ^ 1) * 2 + ds) * 64 + (u + 63)];
                 if (u >= 65) {
                     carry[(tb * 2 + ds) * 64 + (u - 65)] = s;
