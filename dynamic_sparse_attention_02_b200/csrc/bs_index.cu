@@ -63,18 +63,36 @@ struct SmemKeys {
     __device__ uint32_t operator()(int j) const { return float_order_key(p[j]); }
 };
 
-// Shared memory of one CTA: Qm rows [D][kMaxR] and a Km tile [D][kKeyTile],
-// both fp64; scores [R][stride] fp32; one 256-bin histogram per warp.
+// fp64 operand rows in shared memory are padded by 4 doubles, so that the
+// 8 x 4 fragments of one quarter-warp (4 rows x 4 columns) fall in distinct banks.
+template <int D>
+constexpr int bs_row() {
+    return D + 4;
+}
+
+// Shared memory of one CTA: Qm rows [kMaxR][D + 4] and a Km tile
+// [kKeyTile][D + 4], both fp64; scores [R][stride] fp32; one 256-bin
+// histogram per warp.
 template <int D>
 constexpr size_t bs_fixed_smem() {
-    return (size_t)D * kMaxR * 8 + (size_t)D * kKeyTile * 8 + (kTopkThreads / 32) * 256 * 4;
+    return (size_t)kMaxR * bs_row<D>() * 8 + (size_t)kKeyTile * bs_row<D>() * 8 +
+           (kTopkThreads / 32) * 256 * 4;
+}
+
+// D (8 x 8, fp64) += A (8 x 4) B (4 x 8) on the fp64 tensor path; lane l holds
+// A[l / 4][l % 4], B[l % 4][l / 4] and D[l / 4][2 (l % 4) + {0, 1}].
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
 }
 
 // CTA = R consecutive query blocks of one head.
-//  scores: warp w computes rows 2w and 2w+1, lane l key blocks 2l and 2l+1 of
-//          each 64-block tile, as fp64 sums of exact fp32 products over the
-//          d coordinates (operands widened once, on their way into shared
-//          memory); S = scale * sum, rounded to fp32 for ranking.
+//  scores: warp w computes all R (<= 16) rows against key blocks 8w .. 8w+7
+//          of each 64-block tile, as fp64 sums of exact fp32 products over
+//          the d coordinates (operands widened once, on their way into shared
+//          memory; 8 x 8 x 4 fp64 MMAs, two per 4 coordinates);
+//          S = scale * sum, rounded to fp32 for ranking.
 //  top-k:  warp w selects rows w, w + 8, ... by a warp-wide radix select over
 //          its row of S, ties toward the lower block, output ascending.
 template <int D>
@@ -82,10 +100,11 @@ __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     const float* __restrict__ qm, const float* __restrict__ km, int Hq, int Hkv, int nB,
     int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk, RowCounts tk,
     int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt) {
+    constexpr int RS = bs_row<D>();
     extern __shared__ __align__(16) double dsm[];
-    double* Qs = dsm;                          // [D][kMaxR]
-    double* Ks = Qs + D * kMaxR;               // [D][kKeyTile]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + D * kKeyTile);  // [8][256]
+    double* Qs = dsm;                          // [kMaxR][D + 4]
+    double* Ks = Qs + kMaxR * RS;              // [kKeyTile][D + 4]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + kKeyTile * RS);  // [8][256]
     float* S = reinterpret_cast<float*>(hist + (kTopkThreads / 32) * 256);  // [R][stride]
     const int pos = blockIdx.y;
     const int bq0 = blockIdx.x * R;
@@ -101,43 +120,51 @@ __global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
     const float* kmg = km + (size_t)gi * nB * D;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    // consecutive threads fill consecutive shared words (no bank conflicts)
-    for (int t = threadIdx.x; t < kMaxR * D; t += blockDim.x) {
-        const int r = t % kMaxR, c = t / kMaxR;
-        Qs[c * kMaxR + r] = r < nr ? (double)qm[((size_t)pos * nB + bq0 + r) * D + c] : 0.0;
+    // rows widened to fp64 once; rows past nr read 0
+    for (int t = threadIdx.x; t < kMaxR * (D / 4); t += blockDim.x) {
+        const int r = t / (D / 4), c4 = t % (D / 4);
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < nr) f = *reinterpret_cast<const float4*>(qm + ((size_t)pos * nB + bq0 + r) * D + 4 * c4);
+        double* d = Qs + r * RS + 4 * c4;
+        d[0] = f.x;
+        d[1] = f.y;
+        d[2] = f.z;
+        d[3] = f.w;
     }
+    const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
     for (int kt0 = 0; kt0 < ncand; kt0 += kKeyTile) {
         __syncthreads();  // the previous tile has been used
         for (int t = threadIdx.x; t < kKeyTile * (D / 4); t += blockDim.x) {
-            const int kb = t % kKeyTile, c4 = t / kKeyTile;
+            const int kb = t / (D / 4), c4 = t % (D / 4);
             float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
             if (kt0 + kb < ncand)
                 f = *reinterpret_cast<const float4*>(kmg + (size_t)(kt0 + kb) * D + 4 * c4);
-            Ks[(4 * c4 + 0) * kKeyTile + kb] = f.x;
-            Ks[(4 * c4 + 1) * kKeyTile + kb] = f.y;
-            Ks[(4 * c4 + 2) * kKeyTile + kb] = f.z;
-            Ks[(4 * c4 + 3) * kKeyTile + kb] = f.w;
+            double* d = Ks + kb * RS + 4 * c4;
+            d[0] = f.x;
+            d[1] = f.y;
+            d[2] = f.z;
+            d[3] = f.w;
         }
         __syncthreads();
-        if (2 * warp < nr) {
-            double a00 = 0.0, a01 = 0.0, a10 = 0.0, a11 = 0.0;
+        if (kt0 + 8 * warp < ncand) {
+            double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // rows fr, 8 + fr
+            const double* qa = Qs + fr * RS + fc;
+            const double* kbp = Ks + (8 * warp + fr) * RS + fc;
 #pragma unroll 8
-            for (int c = 0; c < D; ++c) {
-                const double2 qv = *reinterpret_cast<const double2*>(Qs + c * kMaxR + 2 * warp);
-                const double2 kv = *reinterpret_cast<const double2*>(Ks + c * kKeyTile + 2 * lane);
-                a00 = fma(qv.x, kv.x, a00);
-                a01 = fma(qv.x, kv.y, a01);
-                a10 = fma(qv.y, kv.x, a10);
-                a11 = fma(qv.y, kv.y, a11);
+            for (int c = 0; c < D; c += 4) {
+                const double b = kbp[c];
+                dmma_8x8x4(c00, c01, qa[c], b);
+                dmma_8x8x4(c10, c11, qa[8 * RS + c], b);
             }
-            const int k0 = kt0 + 2 * lane, r0 = 2 * warp;
-            if (k0 < ncand) {
-                S[r0 * stride + k0] = (float)(a00 * scale);
-                if (r0 + 1 < nr) S[(r0 + 1) * stride + k0] = (float)(a10 * scale);
-            }
-            if (k0 + 1 < ncand) {
-                S[r0 * stride + k0 + 1] = (float)(a01 * scale);
-                if (r0 + 1 < nr) S[(r0 + 1) * stride + k0 + 1] = (float)(a11 * scale);
+            const int k0 = kt0 + 8 * warp + 2 * fc;
+            const double acc[2][2] = {{c00, c01}, {c10, c11}};
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int r = 8 * m + fr;
+                if (r >= nr) continue;
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    if (k0 + e < ncand) S[r * stride + k0 + e] = (float)(acc[m][e] * scale);
             }
         }
     }

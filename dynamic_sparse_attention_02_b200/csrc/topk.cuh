@@ -207,10 +207,21 @@ __device__ void warp_radix_select(const Get& get, int n, int k, uint32_t* hist, 
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int b = lane; b < 256; b += 32) hist[b] = 0;
         __syncwarp();
+        // runs of one bin per lane are counted in a register (see block_radix_select)
+        uint32_t run_bin = 0, run_cnt = 0;
         for (int j = lane; j < n; j += 32) {
             const uint32_t key = get(j);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((key & mask) == prefix) {
+                const uint32_t b = (key >> shift) & 255u;
+                if (run_cnt != 0 && b != run_bin) {
+                    atomicAdd(&hist[run_bin], run_cnt);
+                    run_cnt = 0;
+                }
+                run_bin = b;
+                ++run_cnt;
+            }
         }
+        if (run_cnt != 0) atomicAdd(&hist[run_bin], run_cnt);
         __syncwarp();
         // lane l owns bins 255-8l down to 248-8l; a scan over the lanes gives the
         // count above each lane's bins, so one lane holds the bin where the
