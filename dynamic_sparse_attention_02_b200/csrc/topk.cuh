@@ -53,6 +53,7 @@ struct TopkSmem {
     int warp_tot[33];
     uint32_t prefix;
     int remaining;
+    int done;
 };
 
 // Find threshold key T and the number of keys equal to T to keep, for the
@@ -63,6 +64,7 @@ __device__ void block_radix_select(const Get& get, int n, int k, TopkSmem& s, ui
     if (threadIdx.x == 0) {
         s.prefix = 0;
         s.remaining = k;
+        s.done = 0;
     }
     uint32_t mask = 0;
     for (int shift = 24; shift >= 0; shift -= 8) {
@@ -104,10 +106,19 @@ __device__ void block_radix_select(const Get& get, int n, int k, TopkSmem& s, ui
                 if (c >= rem) break;
                 rem -= c;
             }
-            s.remaining = rem;
-            s.prefix = prefix | ((uint32_t)b << shift);
+            const uint32_t np = prefix | ((uint32_t)b << shift);
+            if ((int)s.hist[b] == rem && np != 0) {
+                // the bin is taken whole: every key >= np, none equal to np - 1
+                s.prefix = np - 1;
+                s.remaining = 0;
+                s.done = 1;
+            } else {
+                s.remaining = rem;
+                s.prefix = np;
+            }
         }
         __syncthreads();
+        if (s.done) break;
         mask |= 255u << shift;
     }
     thr = s.prefix;
@@ -250,11 +261,22 @@ __device__ void warp_radix_select(const Get& get, int n, int k, uint32_t* hist, 
             }
             left -= c[u];
         }
+        int csel = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (255 - 8 * lane - u == bsel) csel = c[u];
         bsel = __shfl_sync(0xffffffffu, bsel, src);
         rem = __shfl_sync(0xffffffffu, left, src);
+        csel = __shfl_sync(0xffffffffu, csel, src);
         prefix |= (uint32_t)bsel << shift;
         mask |= 255u << shift;
         __syncwarp();
+        if (csel == rem && prefix != 0) {
+            // the bin is taken whole: every key >= prefix, none equal to prefix - 1
+            thr = prefix - 1;
+            need_eq = 0;
+            return;
+        }
     }
     thr = prefix;
     need_eq = rem;
