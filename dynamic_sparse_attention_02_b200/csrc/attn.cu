@@ -341,12 +341,14 @@ struct Producer {
             mbar_arrive_expect_tx(&bars.kv_full[st], 2 * L::kKVBytes);
             uint8_t* kd = sm + L::k_off + st * L::kKVBytes;
             uint8_t* vd = sm + L::v_off + st * L::kKVBytes;
+            // every query block of the KV head reads these keys again: keep them in L2
+            const uint64_t pol = l2_policy_evict_last();
 #pragma unroll
             for (int pn = 0; pn < D / 64; ++pn)
-                tma_load_2d(kd + pn * kKVPanel, tmK, 64 * pn, row, &bars.kv_full[st]);
+                tma_load_2d_hint(kd + pn * kKVPanel, tmK, 64 * pn, row, &bars.kv_full[st], pol);
 #pragma unroll
             for (int pn = 0; pn < D / 64; ++pn)
-                tma_load_2d(vd + pn * kKVPanel, tmV, 64 * pn, row, &bars.kv_full[st]);
+                tma_load_2d_hint(vd + pn * kKVPanel, tmV, 64 * pn, row, &bars.kv_full[st], pol);
         }
         __syncwarp();
         ++nkv;
@@ -453,10 +455,11 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
         prefetch_tmap(tmK);
         prefetch_tmap(tmV);
         mbar_arrive_expect_tx(bars.q_full, 2 * L::kQBytes);
+        const uint64_t once = l2_policy_evict_first();  // this CTA's rows, read once
         for (int x = 0; x < 2; ++x)
             for (int pn = 0; pn < D / 64; ++pn)
-                tma_load_2d(sm + L::q_off + x * L::kQBytes + pn * kQPanel, tmQ, 64 * pn,
-                            qh * p.N + 256 * T + 128 * x, bars.q_full);
+                tma_load_2d_hint(sm + L::q_off + x * L::kQBytes + pn * kQPanel, tmQ, 64 * pn,
+                                 qh * p.N + 256 * T + 128 * x, bars.q_full, once);
     }
 
     // per-pattern block map
@@ -904,10 +907,12 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
         for (int u = 0; u < 16; ++u)
             pk[u] = pack_bf16(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
         if (row_ok) {
+            // streaming stores: the output is not read again, so it should not
+            // displace the keys and values other CTAs still read from L2
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                __stcs(dst + u, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
         }
     }
     if (row_ok && p.lse)
