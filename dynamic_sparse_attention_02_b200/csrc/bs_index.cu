@@ -96,7 +96,7 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 //  top-k:  warp w selects rows w, w + 8, ... by a warp-wide radix select over
 //          its row of S, ties toward the lower block, output ascending.
 template <int D>
-__global__ void __launch_bounds__(kTopkThreads) bs_topk_kernel(
+__global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
     const float* __restrict__ qm, const float* __restrict__ km, int Hq, int Hkv, int nB,
     int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk, RowCounts tk,
     int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt) {

@@ -207,6 +207,21 @@ __device__ void block_select_compact(const Get& get, int n, int k, uint32_t thr,
     __syncthreads();
 }
 
+// One key into a run-length histogram count: a run of equal bins is held in
+// (rb, rc) and added to the shared histogram when the bin changes.
+__device__ __forceinline__ void run_count(uint32_t key, uint32_t mask, uint32_t prefix, int shift,
+                                          uint32_t* hist, uint32_t& rb, uint32_t& rc) {
+    if ((key & mask) == prefix) {
+        const uint32_t b = (key >> shift) & 255u;
+        if (rc != 0 && b != rb) {
+            atomicAdd(&hist[rb], rc);
+            rc = 0;
+        }
+        rb = b;
+        ++rc;
+    }
+}
+
 // ---- one warp per selection (many short rows at once), same contract as above.
 // `hist` is this warp's own 256-entry shared histogram.
 template <class Get>
@@ -218,21 +233,27 @@ __device__ void warp_radix_select(const Get& get, int n, int k, uint32_t* hist, 
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int b = lane; b < 256; b += 32) hist[b] = 0;
         __syncwarp();
-        // runs of one bin per lane are counted in a register (see block_radix_select)
-        uint32_t run_bin = 0, run_cnt = 0;
-        for (int j = lane; j < n; j += 32) {
-            const uint32_t key = get(j);
-            if ((key & mask) == prefix) {
-                const uint32_t b = (key >> shift) & 255u;
-                if (run_cnt != 0 && b != run_bin) {
-                    atomicAdd(&hist[run_bin], run_cnt);
-                    run_cnt = 0;
-                }
-                run_bin = b;
-                ++run_cnt;
-            }
+        // runs of one bin are counted in registers (see block_radix_select); each
+        // lane reads four independent streams (keys j = 128 i + 32 t + lane), each
+        // with its own run, so that four load/count chains are in flight at once
+        uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0, c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+        int j0 = 0;
+        for (; j0 + 128 <= n; j0 += 128) {
+            const uint32_t k0 = get(j0 + lane), k1 = get(j0 + 32 + lane);
+            const uint32_t k2 = get(j0 + 64 + lane), k3 = get(j0 + 96 + lane);
+            run_count(k0, mask, prefix, shift, hist, b0, c0);
+            run_count(k1, mask, prefix, shift, hist, b1, c1);
+            run_count(k2, mask, prefix, shift, hist, b2, c2);
+            run_count(k3, mask, prefix, shift, hist, b3, c3);
         }
-        if (run_cnt != 0) atomicAdd(&hist[run_bin], run_cnt);
+        if (j0 + lane < n) run_count(get(j0 + lane), mask, prefix, shift, hist, b0, c0);
+        if (j0 + 32 + lane < n) run_count(get(j0 + 32 + lane), mask, prefix, shift, hist, b1, c1);
+        if (j0 + 64 + lane < n) run_count(get(j0 + 64 + lane), mask, prefix, shift, hist, b2, c2);
+        if (j0 + 96 + lane < n) run_count(get(j0 + 96 + lane), mask, prefix, shift, hist, b3, c3);
+        if (c0 != 0) atomicAdd(&hist[b0], c0);
+        if (c1 != 0) atomicAdd(&hist[b1], c1);
+        if (c2 != 0) atomicAdd(&hist[b2], c2);
+        if (c3 != 0) atomicAdd(&hist[b3], c3);
         __syncwarp();
         // lane l owns bins 255-8l down to 248-8l; a scan over the lanes gives the
         // count above each lane's bins, so one lane holds the bin where the
@@ -288,18 +309,28 @@ __device__ void warp_select_compact(const Get& get, int n, int k, uint32_t thr, 
     const int lane = threadIdx.x & 31;
     const unsigned below = (1u << lane) - 1u;
     int eq_base = 0, sel_base = 0;
-    for (int base = 0; base < n && sel_base < k; base += 32) {
-        const int j = base + lane;
-        const uint32_t key = j < n ? get(j) : 0u;
-        const bool gt = j < n && key > thr;
-        const bool eq = j < n && key == thr;
-        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-        const bool sel = gt || (eq && eq_base + __popc(eqm & below) < need_eq);
-        const unsigned selm = __ballot_sync(0xffffffffu, sel);
-        const int pos = sel_base + __popc(selm & below);
-        if (sel && pos < k) out[pos] = j;
-        eq_base += __popc(eqm);
-        sel_base += __popc(selm);
+    // four 32-key steps per round: their loads are issued together, then the
+    // steps are placed in index order by ballots
+    for (int base = 0; base < n && sel_base < k; base += 128) {
+        uint32_t kb[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int j = base + 32 * t + lane;
+            kb[t] = j < n ? get(j) : 0u;
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int j = base + 32 * t + lane;
+            const bool gt = j < n && kb[t] > thr;
+            const bool eq = j < n && kb[t] == thr;
+            const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+            const bool sel = gt || (eq && eq_base + __popc(eqm & below) < need_eq);
+            const unsigned selm = __ballot_sync(0xffffffffu, sel);
+            const int pos = sel_base + __popc(selm & below);
+            if (sel && pos < k) out[pos] = j;
+            eq_base += __popc(eqm);
+            sel_base += __popc(selm);
+        }
     }
 }
 
