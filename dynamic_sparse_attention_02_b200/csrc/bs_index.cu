@@ -132,20 +132,35 @@ __global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
         d[3] = f.w;
     }
     const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
+    // the key tile is fetched one tile ahead into registers, so that its global
+    // loads are in flight while the MMAs of the current tile run
+    constexpr int kPf = kKeyTile * (D / 4) / kTopkThreads;  // float4 per thread per tile
+    float4 pf[kPf];
+    auto fetch = [&](int kt) {
+#pragma unroll
+        for (int u = 0; u < kPf; ++u) {
+            const int t = threadIdx.x + u * kTopkThreads;
+            const int kb = t / (D / 4), c4 = t % (D / 4);
+            pf[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kt + kb < ncand)
+                pf[u] = *reinterpret_cast<const float4*>(kmg + (size_t)(kt + kb) * D + 4 * c4);
+        }
+    };
+    fetch(0);
     for (int kt0 = 0; kt0 < ncand; kt0 += kKeyTile) {
         __syncthreads();  // the previous tile has been used
-        for (int t = threadIdx.x; t < kKeyTile * (D / 4); t += blockDim.x) {
+#pragma unroll
+        for (int u = 0; u < kPf; ++u) {
+            const int t = threadIdx.x + u * kTopkThreads;
             const int kb = t / (D / 4), c4 = t % (D / 4);
-            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (kt0 + kb < ncand)
-                f = *reinterpret_cast<const float4*>(kmg + (size_t)(kt0 + kb) * D + 4 * c4);
             double* d = Ks + kb * RS + 4 * c4;
-            d[0] = f.x;
-            d[1] = f.y;
-            d[2] = f.z;
-            d[3] = f.w;
+            d[0] = pf[u].x;
+            d[1] = pf[u].y;
+            d[2] = pf[u].z;
+            d[3] = pf[u].w;
         }
         __syncthreads();
+        if (kt0 + kKeyTile < ncand) fetch(kt0 + kKeyTile);
         if (kt0 + 8 * warp < ncand) {
             double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // rows fr, 8 + fr
             const double* qa = Qs + fr * RS + fc;
