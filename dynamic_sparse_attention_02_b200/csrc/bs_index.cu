@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kPoolThreads) meanpool_kernel(const bf16* __re
 }
 
 constexpr int kMaxR = 16;       // query-block rows per CTA (fewer when the rows are long)
-constexpr int kTopkThreads = 256;
+constexpr int kTopkThreads = 512;
 constexpr int kKeyTile = 64;     // key blocks per shared-memory tile
 constexpr size_t kBsSmemCap = 227 * 1024;
 
@@ -88,12 +88,12 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 }
 
 // CTA = R consecutive query blocks of one head.
-//  scores: warp w computes all R (<= 16) rows against key blocks 8w .. 8w+7
-//          of each 64-block tile, as fp64 sums of exact fp32 products over
-//          the d coordinates (operands widened once, on their way into shared
-//          memory; 8 x 8 x 4 fp64 MMAs, two per 4 coordinates);
+//  scores: 16 warps; warp w computes rows 8 (w / 8) .. +7 against key blocks
+//          8 (w % 8) .. +7 of each 64-block tile, as fp64 sums of exact fp32
+//          products over the d coordinates (operands widened once, on their way
+//          into shared memory; one 8 x 8 x 4 fp64 MMA per 4 coordinates);
 //          S = scale * sum, rounded to fp32 for ranking.
-//  top-k:  warp w selects rows w, w + 8, ... by a warp-wide radix select over
+//  top-k:  warp w selects rows w, w + 16, ... by a warp-wide radix select over
 //          its row of S, ties toward the lower block, output ascending.
 template <int D>
 __global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
@@ -161,25 +161,19 @@ __global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
         }
         __syncthreads();
         if (kt0 + kKeyTile < ncand) fetch(kt0 + kKeyTile);
-        if (kt0 + 8 * warp < ncand) {
-            double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // rows fr, 8 + fr
-            const double* qa = Qs + fr * RS + fc;
-            const double* kbp = Ks + (8 * warp + fr) * RS + fc;
+        // warp w: rows 8 (w / 8) .. +7 against key blocks 8 (w % 8) .. +7 of the tile
+        const int mt = warp >> 3, kg = warp & 7;
+        if (kt0 + 8 * kg < ncand && 8 * mt < nr) {
+            double c0 = 0.0, c1 = 0.0;
+            const double* qa = Qs + (8 * mt + fr) * RS + fc;
+            const double* kbp = Ks + (8 * kg + fr) * RS + fc;
 #pragma unroll 8
-            for (int c = 0; c < D; c += 4) {
-                const double b = kbp[c];
-                dmma_8x8x4(c00, c01, qa[c], b);
-                dmma_8x8x4(c10, c11, qa[8 * RS + c], b);
-            }
-            const int k0 = kt0 + 8 * warp + 2 * fc;
-            const double acc[2][2] = {{c00, c01}, {c10, c11}};
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int r = 8 * m + fr;
-                if (r >= nr) continue;
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    if (k0 + e < ncand) S[r * stride + k0 + e] = (float)(acc[m][e] * scale);
+            for (int c = 0; c < D; c += 4) dmma_8x8x4(c0, c1, qa[c], kbp[c]);
+            const int k0 = kt0 + 8 * kg + 2 * fc;
+            const int r = 8 * mt + fr;
+            if (r < nr) {
+                if (k0 < ncand) S[r * stride + k0] = (float)(c0 * scale);
+                if (k0 + 1 < ncand) S[r * stride + k0 + 1] = (float)(c1 * scale);
             }
         }
     }
