@@ -30,6 +30,7 @@
 // TMEM (512 columns): slot x owns [256x, 256x+256): S buffers 0 and 1 at
 // +0 and +64 (64 columns each; P, bf16 pairs, reuses the first 32), O at
 // +128 (d columns).
+#include <atomic>
 #include <cfloat>
 #include <cstring>
 #include <cudaTypedefs.h>
@@ -1107,10 +1108,12 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
         !make_tma_map(&tmK, a.k, (long long)a.Hkv * a.N, D, 64) ||
         !make_tma_map(&tmV, a.v, (long long)a.Hkv * a.N, D, 64))
         return cudaErrorInvalidValue;
-    static unsigned int seq = 0;
+    // launch sequence number (never 0), unique across host threads
+    static std::atomic<unsigned int> next_seq{0};
+    unsigned int seq = ++next_seq;
     AttnParams p;
     memset(&p, 0, sizeof(p));
-    if (++seq == 0) ++seq;
+    if (seq == 0) seq = ++next_seq;
     p.seq = seq;
     p.k = a.k;
     p.v = a.v;

@@ -27,6 +27,7 @@
 // rows: warp w reads lane quadrant w % 4, and the epilogue warps of one
 // quadrant split the tile's 128 key columns between them.  Two 128-column accumulators let the tensor core fill one while
 // the epilogue drains the other.
+#include <atomic>
 #include <cfloat>
 
 #include "internal.h"
@@ -619,10 +620,12 @@ cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, 
     if (!make_tma_map(&tmQ, q, (long long)Hq * N, d, 64) ||
         !make_tma_map(&tmK, k, (long long)Hkv * N, d, kTcKeys))
         return cudaErrorInvalidValue;
-    static unsigned int seq = 0;
+    // launch sequence number (never 0), unique across host threads
+    static std::atomic<unsigned int> next_seq{0};
+    unsigned int seq = ++next_seq;
     TcParams p;
     memset(&p, 0, sizeof(p));
-    if (++seq == 0) ++seq;
+    if (seq == 0) seq = ++next_seq;
     p.seq = seq;
     p.heads = heads;
     // pair the listed heads of each KV head in list order; an odd one out runs alone
