@@ -30,7 +30,7 @@
  *  - same guide, "Vertical-Slash Kernel Mechanics": online-softmax attention
  *    over only the selected entries.
  *
- * Readings where the pages leave a step open (each also listed in the design doc):
+ * Readings where the pages leave a step open:
  *  - softmax scale is 1/sqrt(d) (guide, "Calibration Forward Pass");
  *  - Vertical-Slash index: row softmax over the causal keys j <= i of each
  *    of the last `last_q` rows, summed per column j (vertical) and per

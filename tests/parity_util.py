@@ -4,7 +4,7 @@ import torch
 
 import oracle
 
-# spec tolerances for bf16 attention output against the oracle
+# required accuracy of the bf16 attention output against the oracle
 ATTN_MAX_ABS = 1e-2
 ATTN_MEAN_ABS = 1e-3
 # index sets may differ only at entries within this relative distance of the k-th score
@@ -48,7 +48,7 @@ def check_index_set(gpu_idx, scores, k, window_scale=None, what=""):
 
 
 def check_attn(out_gpu, lse_gpu, out_ref, lse_ref, what=""):
-    """bf16 GPU rows against fp64 oracle rows: spec max / mean abs error."""
+    """bf16 GPU rows against fp64 oracle rows: max-abs <= 1e-2 and mean-abs <= 1e-3."""
     o = out_gpu.float().cpu().numpy().astype(np.float64)
     err = np.abs(o - out_ref)
     assert np.all(np.isfinite(o)), f"{what}: non-finite output"

@@ -4,7 +4,7 @@ against the CPU oracle on seeded heads and rows it can compute one by one.
 
 For each sampled head: the GPU index sets must equal the oracle's except
 within the tie window of the k-th score; the GPU attention fed the oracle's
-own indices must meet the spec error bounds on the sampled rows; and
+own indices must meet max-abs <= 1e-2, mean-abs <= 1e-3 on the sampled rows; and
 where the GPU's index equals the oracle's exactly, the layer's own output at
 those rows must too.
 """

@@ -54,7 +54,7 @@ def test_dense_matches_sdpa(Hq, Hkv, N, d):
 
 
 def test_full_budgets_reduce_to_dense():
-    """Budgets that cover everything give dense causal attention (spec pin)."""
+    """Budgets that cover everything give dense causal attention."""
     Hq, Hkv, N, d = 2, 1, 256, 64
     q, k, v = rand_qkv(Hq, Hkv, N, d, 2)
     ref = sdpa_rows(q, k, v, 1, causal=True)
