@@ -20,36 +20,48 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 
+// One 64-row block per warp: lane l reads 16-byte column chunk l % (D/8) of
+// the rows of its row group (64 / (32 / (D/8)) rows), eight loads in flight,
+// sums them in fp64 (exact), and the row groups meet by shuffles.
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) meanpool_kernel(const bf16* __restrict__ x,
                                                                 int N, int nB, HeadList items,
                                                                 float* __restrict__ out) {
-    constexpr int kCPR = D / 8;                 // 16-byte chunks per row
-    constexpr int kRG = kPoolThreads / kCPR;    // row groups
-    constexpr int kRows = 64 / kRG;             // rows per thread
-    __shared__ double red[kRG * D];
-    const int b = blockIdx.x, item = blockIdx.y;
+    constexpr int kCPR = D / 8;          // 16-byte chunks per row
+    constexpr int kGroups = 32 / kCPR;   // row groups per warp
+    constexpr int kRows = 64 / kGroups;  // rows per lane
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int b = blockIdx.x * (kPoolThreads / 32) + warp, item = blockIdx.y;
+    if (b >= nB) return;
     const int hd = head_qh(items.e[item]);
-    const bf16* base = x + ((long long)hd * N + (long long)b * 64) * D;
-    const int c = threadIdx.x % kCPR, rg = threadIdx.x / kCPR;
+    const int c = lane % kCPR, grp = lane / kCPR;
+    const bf16* base = x + ((long long)hd * N + (long long)b * 64 + grp * kRows) * D + c * 8;
     double acc[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = 0.0;
+    for (int v = 0; v < 8; ++v) acc[v] = 0.0;
 #pragma unroll
-    for (int u = 0; u < kRows; ++u) {
-        const int r = rg + u * kRG;
-        const uint4 raw = *reinterpret_cast<const uint4*>(base + (long long)r * D + c * 8);
-        const bf16* e = reinterpret_cast<const bf16*>(&raw);
+    for (int r0 = 0; r0 < kRows; r0 += 8) {
+        uint4 raw[8];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) acc[v] += (double)__bfloat162float(e[v]);
+        for (int u = 0; u < 8; ++u)
+            raw[u] = *reinterpret_cast<const uint4*>(base + (long long)(r0 + u) * D);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bf16* e = reinterpret_cast<const bf16*>(&raw[u]);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[v] += (double)__bfloat162float(e[v]);
+        }
     }
 #pragma unroll
-    for (int v = 0; v < 8; ++v) red[rg * D + c * 8 + v] = acc[v];
-    __syncthreads();
-    for (int col = threadIdx.x; col < D; col += blockDim.x) {
-        double s = 0.0;
-        for (int g = 0; g < kRG; ++g) s += red[g * D + col];
-        out[((size_t)item * nB + b) * D + col] = (float)(s / 64.0);
+    for (int off = kCPR; off < 32; off <<= 1)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], off);
+    if (grp == 0) {
+        float4* o = reinterpret_cast<float4*>(out + ((size_t)item * nB + b) * D + c * 8);
+        o[0] = make_float4((float)(acc[0] / 64.0), (float)(acc[1] / 64.0), (float)(acc[2] / 64.0),
+                           (float)(acc[3] / 64.0));
+        o[1] = make_float4((float)(acc[4] / 64.0), (float)(acc[5] / 64.0), (float)(acc[6] / 64.0),
+                           (float)(acc[7] / 64.0));
     }
 }
 
@@ -220,8 +232,9 @@ cudaError_t launch_bs_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, do
     for (int i = 0; i < heads.n; ++i) used[kv_head_of(head_qh(heads.e[i]), Hq, Hkv)] = true;
     for (int g = 0; g < Hkv; ++g)
         if (used[g]) kvs.e[kvs.n++] = pack_head(g, 0, 0);
-    meanpool_kernel<D><<<dim3(nB, heads.n), kPoolThreads, 0, st>>>(q, N, nB, heads, ws.qm);
-    meanpool_kernel<D><<<dim3(nB, kvs.n), kPoolThreads, 0, st>>>(k, N, nB, kvs, ws.km);
+    const int pool_x = (nB + kPoolThreads / 32 - 1) / (kPoolThreads / 32);
+    meanpool_kernel<D><<<dim3(pool_x, heads.n), kPoolThreads, 0, st>>>(q, N, nB, heads, ws.qm);
+    meanpool_kernel<D><<<dim3(pool_x, kvs.n), kPoolThreads, 0, st>>>(k, N, nB, kvs, ws.km);
     RowCounts tk{};
     if (topk_rows) {
         tk.n = heads.n;
