@@ -56,15 +56,15 @@ struct WsCarver {
 };
 
 // ----------------------------------------------------------- VS index
-constexpr int kVsChunk = 1024;  // keys per CTA in the score passes
-
 struct VsIndexWs {
-    double* m_part;  // [n_heads][L][nchunks]
+    double* m_part;  // [n_heads][L][ceil(N / kVsTcChunk)]
     double* l_part;
     double* mrow;    // [n_heads][L] merged row max
     double* linv;    // [n_heads][L] 1 / merged row sum
     float* vscore;   // [n_heads][N]
     float* sscore;   // [n_heads][N]
+    float* vpart;    // [n_heads][ceil(L / 64)][N] partial scores (L > 64 only, else null)
+    float* spart;
 };
 VsIndexWs carve_vs_index(WsCarver& c, int n_heads, int N, int L, bool need_vscore,
                          bool need_sscore);
@@ -76,10 +76,11 @@ cudaError_t launch_vs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N
                             const VsIndexWs& ws, cudaStream_t st,
                             const int32_t* kv_rows = nullptr, const int32_t* ks_rows = nullptr);
 
-// The two score passes on the tensor cores, for L <= 64 (vs_score_tc.cu).
+// The two score passes on the tensor cores (vs_score_tc.cu), any L <= 1024.
 // Pass 1 writes ws.m_part / ws.l_part for chunks of kVsTcChunk keys (merge
 // them with nchunks = ceil(N / kVsTcChunk)); pass 2 reads ws.mrow / ws.linv
-// and writes every entry of vscore / sscore [n_heads][N].
+// and writes every entry of vscore / sscore [n_heads][N] (through
+// ws.vpart / ws.spart when L > 64).
 constexpr int kVsTcChunk = 2048;
 cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, int Hkv, int N,
                                 int d, double scale, int L, const HeadList& heads,

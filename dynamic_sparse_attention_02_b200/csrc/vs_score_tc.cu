@@ -1,32 +1,35 @@
-// vs_score_tc.cu -- the Vertical-Slash score passes on the tensor cores
-// (last_q <= 64).
+// vs_score_tc.cu -- the Vertical-Slash score passes on the tensor cores.
 //
 // MInference 1.0 (hotpaper.ai summary, "key idea"; guide "2. The
 // Vertical-Slash Pattern"): the last L queries of a head score every key
 // column and every diagonal through their causal row softmax.  The products
-// q_i . k_j form a dense contraction, so here they run on tcgen05: one M=128
-// tile stacks the last 64 query rows of two query heads that share a KV head
-// (rows 0-63 the first head, 64-127 the second; for L < 64 the first 64-L
-// rows of each half are padding), and every 128-key tile of K gives
-// S = Q K^T in TMEM (exact bf16 products, fp32 accumulation).
+// q_i . k_j form a dense contraction, so here they run on tcgen05.  The L rows
+// of a head split into 64-row groups counted from the end (the first group
+// padded when 64 does not divide L); one M=128 tile stacks two such groups of
+// query heads that share a KV head (rows 0-63 the first, 64-127 the second),
+// and every 128-key tile of K gives S = Q K^T in TMEM (exact bf16 products,
+// fp32 accumulation).
 //
 //   pass 1: per row, the online max and sum of exp over a 2048-key chunk
 //           (exponentials in fp32, the running sum in fp64).  The partials go
-//           to the workspace the CUDA-core passes fill and are merged by
-//           vs_rowmerge into each row's max m_i and 1 / l_i.
+//           to the workspace and are merged by vs_rowmerge into each row's
+//           max m_i and 1 / l_i.
 //   pass 2: p_ij = exp(s_ij - m_i) / l_i with the exponent carried as an
 //           unevaluated pair of fp32 values (exp2 of the leading part times a
 //           first-order correction for the rest), staged in shared memory as
 //           fp32 and summed per column and per diagonal with compensated
 //           (Kahan) fp32 sums in a fixed order.  A chunk owns the
 //           columns it holds and the diagonals whose first key it holds, and
-//           reads one more key tile to finish those diagonals.
+//           reads one more key tile to finish those diagonals.  With one row
+//           group per head (L <= 64) these are the scores; otherwise each
+//           group's sums are partials, added per head in group order.
 //
 // Warp roles: warp 0 loads Q and K tiles by TMA, warp 1 issues the MMAs,
 // warps 2.. are the epilogue (8 in pass 1, 16 in pass 2).  TMEM lanes are
 // rows: warp w reads lane quadrant w % 4, and the epilogue warps of one
-// quadrant split the tile's 128 key columns between them.  Two 128-column accumulators let the tensor core fill one while
-// the epilogue drains the other.
+// quadrant split the tile's 128 key columns between them.  Two 128-column
+// accumulators let the tensor core fill one while the epilogue drains the
+// other.
 #include <atomic>
 #include <cfloat>
 
@@ -80,15 +83,17 @@ __device__ __forceinline__ void vs_set_abort(volatile int* abort, unsigned int s
     atomicExch(&g_vs_abort_seq, seq);
 }
 
-// Two listed query heads of one KV head per tile; slot 1 may be empty (-1).
-struct PairList {
-    int n;
-    int16_t pos[2][MI_MAX_HEADS];
-};
-
+// Work items are 64-row groups of the listed heads' last L rows, counted from
+// the end: item = position * G + g (G = ceil(L / 64)) covers the query rows
+// N - 64 (g + 1) .. N - 64 g - 1, those before N - L being padding.  The
+// items of one KV head are paired into M=128 tiles in order (an odd one out
+// runs alone), tile by tile across the KV heads in use.
 struct TcParams {
     HeadList heads;
-    PairList pairs;
+    int16_t hpos[MI_MAX_HEADS];        // listed positions, grouped by KV head
+    int16_t hstart[MI_MAX_HEADS + 1];  // per KV head in use: its first entry in hpos
+    int tstart[MI_MAX_HEADS + 1];      // per KV head in use: its first tile
+    int ngroups, G;
     int Hq, Hkv, N, L, nchunks, chunk;
     double scale;
     unsigned int seq;
@@ -96,9 +101,32 @@ struct TcParams {
     double* l_part;
     const double* mrow;  // pass 2 in: [n_heads][L]
     const double* linv;
-    float* vscore;  // pass 2 out: [n_heads][N]
-    float* sscore;
+    float* vout;  // pass 2 out: [items][N], the scores themselves when G == 1
+    float* sout;  // (items == heads then), else per-item partial sums
 };
+
+// An item's head position, its rows' end e (exclusive), the first non-padding
+// row rmin of its 64 and the index among the head's L rows of its row 0.
+struct TcItem {
+    int item, pos, e, rmin, rbase;
+};
+__device__ __forceinline__ TcItem tc_item(const TcParams& p, int item) {
+    TcItem x;
+    x.item = item;
+    if (item < 0) {
+        x.pos = -1;
+        x.e = 0;
+        x.rmin = 64;
+        x.rbase = 0;
+        return x;
+    }
+    const int g = item % p.G;
+    x.pos = item / p.G;
+    x.e = p.N - 64 * g;
+    x.rbase = p.L - 64 * (g + 1);
+    x.rmin = x.rbase < 0 ? -x.rbase : 0;
+    return x;
+}
 
 // Epilogue width per pass: pass 1 runs two CTAs per SM with 8 epilogue warps
 // (64 key columns each), pass 2 one CTA per SM with 16 (32 columns each), so
@@ -154,15 +182,16 @@ struct TcBars {
 template <int D>
 __device__ void tc_producer(const TcParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                             uint8_t* sm, const TcBars& bars, volatile int* abort, int g, int jb,
-                            int ntiles, int pos_a, int pos_b) {
+                            int ntiles, int it_a, int it_b) {
     using Lay = TcLayout<D, 1>;
     prefetch_tmap(tmQ);
     prefetch_tmap(tmK);
-    const int nslots = pos_b >= 0 ? 2 : 1;
+    const int nslots = it_b >= 0 ? 2 : 1;
     mbar_arrive_expect_tx(bars.q_full, (uint32_t)(nslots * Lay::kPanels * 64 * 128));
     for (int s = 0; s < nslots; ++s) {
-        const int qh = head_qh(p.heads.e[s ? pos_b : pos_a]);
-        const int row = qh * p.N + p.N - 64;
+        const TcItem x = tc_item(p, s ? it_b : it_a);
+        const int qh = head_qh(p.heads.e[x.pos]);
+        const int row = qh * p.N + x.e - 64;
         for (int pn = 0; pn < Lay::kPanels; ++pn)
             tma_load_2d(sm + Lay::q_off + pn * Lay::kQPanel + s * 64 * 128, tmQ, 64 * pn, row,
                         bars.q_full);
@@ -347,7 +376,7 @@ __device__ __forceinline__ int run_valid(bool valid_row, long long i, long long 
 template <int D, int PASS>
 __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                             volatile int* abort, uint32_t tmem, int jb, int je, int ntiles,
-                            int pos_a, int pos_b, int chunk) {
+                            int it_a, int it_b, int chunk) {
     using Lay = TcLayout<D, PASS>;
     using Sh = TcShape<PASS>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -355,11 +384,12 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
     const int quad = warp & 3, grp = (warp - kEpiWarp0) >> 2;
     const int row = 32 * quad + lane;  // tile row = TMEM lane
     const int slot = row >> 6, r = row & 63;
-    const int pos = slot ? pos_b : pos_a;
-    const int L = p.L, N = p.N, rmin = 64 - L;
+    const TcItem me = tc_item(p, slot ? it_b : it_a);
+    const int pos = me.pos;
+    const int L = p.L, N = p.N, rmin = me.rmin;
     const bool valid_row = pos >= 0 && r >= rmin;
-    const long long i = (long long)N - 64 + r;  // this row's query position
-    const int rr = r - rmin;                     // its index among the L rows
+    const long long i = (long long)me.e - 64 + r;  // this row's query position
+    const int rr = me.rbase + r;                     // its index among the L rows
     const uint32_t t_row = tmem + ((uint32_t)(32 * quad) << 16) + Sh::kCols * grp;
     bool failed = false;
 
@@ -480,9 +510,9 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
             for (int rd = et; rd < 256 + 2 * kDiag; rd += Sh::kEpiThreads) {
                 if (rd < 256) {
                     const int cs = rd >> 7, cc = rd & 127;
-                    const int cpos = cs ? pos_b : pos_a;
+                    const int citem = cs ? it_b : it_a;
                     const long long j = j0 + cc;
-                    if (cpos < 0 || j < jb || j >= je) continue;
+                    if (citem < 0 || j < jb || j >= je) continue;
                     const float* col = P + cs * 64 * kSkew + cc + 63;  // row q at q * (kSkew - 1)
                     KahanSum2 ks[2];  // four independent chains (rows q mod 4) in two pairs
 #pragma unroll
@@ -492,14 +522,14 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                             ks[w].add(pk2(col[(q + 2 * w) * (kSkew - 1)],
                                           col[(q + 2 * w + 1) * (kSkew - 1)]));
                     }
-                    p.vscore[(size_t)cpos * N + j] = (float)(ks[0].value() + ks[1].value());
+                    p.vout[(size_t)citem * N + j] = (float)(ks[0].value() + ks[1].value());
                     continue;
                 }
                 const int dd = rd - 256;
                 const int ds = dd >= kDiag ? 1 : 0;
                 const int u = dd - ds * kDiag - 63;
-                const int dpos = ds ? pos_b : pos_a;
-                if (dpos < 0) continue;
+                const TcItem dx = tc_item(p, ds ? it_b : it_a);
+                if (dx.item < 0) continue;
                 const float* dcol = P + ds * 64 * kSkew + u + 63;  // row q at q * kSkew
                 KahanSum2 ks[2];  // four chains in two pairs; positions past a row's keys hold 0
 #pragma unroll
@@ -514,10 +544,10 @@ __device__ void tc_epilogue(const TcParams& p, uint8_t* sm, const TcBars& bars,
                     carry[(tb * 2 + ds) * 64 + (u - 65)] = s;
                     continue;
                 }
-                const long long o = (long long)N - 64 - j0 - u;
+                const long long o = (long long)dx.e - 64 - j0 - u;
                 if (o < 0 || o >= N) continue;
-                const long long fk = max(0LL, j0 + u + rmin);  // the diagonal's first key
-                if (fk >= jb && fk < je) p.sscore[(size_t)dpos * N + o] = (float)s;
+                const long long fk = max(0LL, j0 + u + dx.rmin);  // the diagonal's first key
+                if (fk >= jb && fk < je) p.sout[(size_t)dx.item * N + o] = (float)s;
             }
         }
         epi_bar<PASS>();  // the staging buffer is free again
@@ -545,9 +575,14 @@ __global__ void __launch_bounds__(TcShape<PASS>::kThreads, PASS == 1 ? 2 : 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::misc_off);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + Lay::misc_off + 4);
 
-    const int pair = blockIdx.x, chunk = blockIdx.y;
-    const int pos_a = p.pairs.pos[0][pair], pos_b = p.pairs.pos[1][pair];
-    const int g = kv_head_of(head_qh(p.heads.e[pos_a]), p.Hq, p.Hkv);
+    const int tile = blockIdx.x, chunk = blockIdx.y;
+    int gi = 0;
+    while (gi + 1 < p.ngroups && tile >= p.tstart[gi + 1]) ++gi;
+    const int h0 = p.hstart[gi], nit = (p.hstart[gi + 1] - h0) * p.G;
+    const int k0 = 2 * (tile - p.tstart[gi]);
+    const int it_a = p.hpos[h0 + k0 / p.G] * p.G + k0 % p.G;
+    const int it_b = k0 + 1 < nit ? p.hpos[h0 + (k0 + 1) / p.G] * p.G + (k0 + 1) % p.G : -1;
+    const int g = kv_head_of(head_qh(p.heads.e[it_a / p.G]), p.Hq, p.Hkv);
     const int jb = chunk * p.chunk;
     const int je = min(p.N, jb + p.chunk);
     const int jend = PASS == 1 ? je : min(p.N, je + kTcKeys);
@@ -582,17 +617,35 @@ __global__ void __launch_bounds__(TcShape<PASS>::kThreads, PASS == 1 ? 2 : 1)
 
     if (warp == 0) {
         if ((threadIdx.x & 31) == 0)
-            tc_producer<D>(p, &tmQ, &tmK, sm, bars, abort, g, jb, ntiles, pos_a, pos_b);
+            tc_producer<D>(p, &tmQ, &tmK, sm, bars, abort, g, jb, ntiles, it_a, it_b);
     } else if (warp == 1) {
         tc_mma<D>(p, sm, bars, abort, tmem, ntiles);
         tc_fence_before();
     } else {
-        tc_epilogue<D, PASS>(p, sm, bars, abort, tmem, jb, je, ntiles, pos_a, pos_b, chunk);
+        tc_epilogue<D, PASS>(p, sm, bars, abort, tmem, jb, je, ntiles, it_a, it_b, chunk);
     }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTcTmemCols);
+    }
+}
+
+// last_q > 64: a head's scores are the sums of its items' partial sums, in row
+// group order.  Row group g has no row at or past key (or diagonal) N - 64 g,
+// so its partials there are never written and not read.
+__global__ void vs_part_merge_kernel(const float* __restrict__ vpart,
+                                     const float* __restrict__ spart, int G, int N,
+                                     float* __restrict__ vscore, float* __restrict__ sscore) {
+    const int pos = blockIdx.y;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < N; j += gridDim.x * blockDim.x) {
+        double v = 0.0, sl = 0.0;
+        for (int g = 0; g < G && j < N - 64 * g; ++g) {
+            v += vpart[((size_t)pos * G + g) * N + j];
+            sl += spart[((size_t)pos * G + g) * N + j];
+        }
+        vscore[(size_t)pos * N + j] = (float)v;
+        sscore[(size_t)pos * N + j] = (float)sl;
     }
 }
 
@@ -603,8 +656,8 @@ cudaError_t launch_pass(const CUtensorMap& tmQ, const CUtensorMap& tmK, const Tc
     cudaError_t e = cudaFuncSetAttribute(vs_score_tc_kernel<D, PASS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    vs_score_tc_kernel<D, PASS>
-        <<<dim3(p.pairs.n, p.nchunks), TcShape<PASS>::kThreads, smem, st>>>(tmQ, tmK, p);
+    vs_score_tc_kernel<D, PASS><<<dim3(p.tstart[p.ngroups], p.nchunks), TcShape<PASS>::kThreads,
+                                  smem, st>>>(tmQ, tmK, p);
     return cudaGetLastError();
 }
 
@@ -615,7 +668,7 @@ cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, 
                                 const VsIndexWs& ws, float* vscore, float* sscore,
                                 cudaStream_t st) {
     if (heads.n == 0) return cudaSuccess;
-    if (L < 1 || L > 64 || N < 64 || (d != 64 && d != 128)) return cudaErrorInvalidValue;
+    if (L < 1 || L > N || L > 1024 || N < 64 || (d != 64 && d != 128)) return cudaErrorInvalidValue;
     CUtensorMap tmQ, tmK;
     if (!make_tma_map(&tmQ, q, (long long)Hq * N, d, 64) ||
         !make_tma_map(&tmK, k, (long long)Hkv * N, d, kTcKeys))
@@ -628,28 +681,25 @@ cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, 
     if (seq == 0) seq = ++next_seq;
     p.seq = seq;
     p.heads = heads;
-    // pair the listed heads of each KV head in list order; an odd one out runs alone
-    int np = 0;
+    // items of each KV head in list order (each head's row groups together),
+    // paired into tiles; an odd one out runs alone
+    const int G = (L + 63) / 64;
+    int nh = 0, ng = 0, nt = 0;
     for (int g = 0; g < Hkv; ++g) {
-        int pend = -1;
-        for (int i = 0; i < heads.n; ++i) {
-            if (kv_head_of(head_qh(heads.e[i]), Hq, Hkv) != g) continue;
-            if (pend < 0) {
-                pend = i;
-            } else {
-                p.pairs.pos[0][np] = (int16_t)pend;
-                p.pairs.pos[1][np] = (int16_t)i;
-                ++np;
-                pend = -1;
-            }
-        }
-        if (pend >= 0) {
-            p.pairs.pos[0][np] = (int16_t)pend;
-            p.pairs.pos[1][np] = -1;
-            ++np;
+        const int start = nh;
+        for (int i = 0; i < heads.n; ++i)
+            if (kv_head_of(head_qh(heads.e[i]), Hq, Hkv) == g) p.hpos[nh++] = (int16_t)i;
+        if (nh > start) {
+            p.hstart[ng] = (int16_t)start;
+            p.tstart[ng] = nt;
+            nt += ((nh - start) * G + 1) / 2;
+            ++ng;
         }
     }
-    p.pairs.n = np;
+    p.hstart[ng] = (int16_t)nh;
+    p.tstart[ng] = nt;
+    p.ngroups = ng;
+    p.G = G;
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.N = N;
@@ -661,11 +711,17 @@ cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, 
     p.l_part = ws.l_part;
     p.mrow = ws.mrow;
     p.linv = ws.linv;
-    p.vscore = vscore;
-    p.sscore = sscore;
+    p.vout = G == 1 ? vscore : ws.vpart;
+    p.sout = G == 1 ? sscore : ws.spart;
+    if (G > 1 && (!ws.vpart || !ws.spart)) return cudaErrorInvalidValue;
     if (pass == 1)
         return d == 128 ? launch_pass<128, 1>(tmQ, tmK, p, st) : launch_pass<64, 1>(tmQ, tmK, p, st);
-    return d == 128 ? launch_pass<128, 2>(tmQ, tmK, p, st) : launch_pass<64, 2>(tmQ, tmK, p, st);
+    cudaError_t e = d == 128 ? launch_pass<128, 2>(tmQ, tmK, p, st)
+                             : launch_pass<64, 2>(tmQ, tmK, p, st);
+    if (e != cudaSuccess || G == 1) return e;
+    vs_part_merge_kernel<<<dim3((N + 255) / 256, heads.n), 256, 0, st>>>(ws.vpart, ws.spart, G, N,
+                                                                          vscore, sscore);
+    return cudaGetLastError();
 }
 
 cudaError_t read_vs_wait_failure(int* out8) {
