@@ -133,11 +133,9 @@ size_t mi_prefill_workspace_bytes(int Hq, int Hkv, int N, int d, const int8_t* p
  * Pattern").  For each listed head h and each of the last L = last_q rows
  * i = N-L .. N-1: row softmax of scale * q_i . k_j over j <= i; vertical[j]
  * sums the probabilities of column j over the L rows, slash[o] sums those of
- * diagonal o = i - j.  For last_q <= 64 the products q_i . k_j run on the
- * tensor cores (exact bf16 products, fp32 accumulation; the softmax argument
- * and the sums in fp64, the exponentials as fp32 exp2 with an fp64
- * correction); for larger last_q everything is fp64 on CUDA cores.  Scores
- * are ranked as fp32.
+ * diagonal o = i - j.  The products q_i . k_j run on the tensor cores (exact
+ * bf16 products, fp32 accumulation); the softmax argument and the column and
+ * diagonal sums are carried to fp64 accuracy.  Scores are ranked as fp32.
  * The top vertical_size columns and top slash_size diagonals (ties: lower
  * index first) are written sorted ascending:
  *   v_idx [n_heads][vertical_size], s_idx [n_heads][slash_size] (int32,
