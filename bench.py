@@ -335,9 +335,10 @@ def run_minfer(args):
     n_vs = int(np.sum(pattern == synth.PATTERN_VS))
     n_bs = int(np.sum(pattern == synth.PATTERN_BS))
     # VS: two score passes, the row merge, one top-k launch for both lists, the
-    # slash/vertical prep (last_q > 64 would add nothing: same count);
+    # slash/vertical prep, and for last_q > 64 the merge of row-group partials;
     # BS: mean-pool of Q, of K, block score + top-k; then one attention launch
-    launches_per_step = (4 + 1 if n_vs else 0) + (3 if n_bs else 0) + 1
+    n_vs_launches = 5 + (1 if w.last_q > 64 else 0)
+    launches_per_step = (n_vs_launches if n_vs else 0) + (3 if n_bs else 0) + 1
 
     def step(ev):
         B.mi_prefill_layer(q, k, v, pattern, params, out=out, ws=ws, stage_events=ev)
