@@ -5,12 +5,12 @@
 // 64-token blocks, each query block scores every causal key block by the
 // dot product of the pooled vectors, and the top-k key blocks are kept.
 //
-//   meanpool:  Qm[h][b] = mean of q rows 64b..64b+63 (fp64 sum, fp32 out),
+//   meanpool:  Qm[h][b] = mean of q rows 64b..64b+63 (fp64, exact),
 //              Km[g][b] likewise.  Pure HBM stream with 16-byte loads.
-//   bs_topk:   S[bq][bk] = scale * Qm[bq] . Km[bk] for bk <= bq (fp64 sum of
-//              exact fp32 products, ranked as fp32), register-tiled and kept
-//              on chip, then a warp-wide radix top-k per query block,
-//              ascending output.
+//   bs_topk:   S[bq][bk] = scale * Qm[bq] . Km[bk] for bk <= bq (fp64 dot
+//              products on the fp64 tensor path, ranked as fp32), kept on
+//              chip, then a warp-wide radix top-k per query block, ascending
+//              output.
 #include "internal.h"
 #include "topk.cuh"
 
@@ -26,7 +26,7 @@ constexpr int kPoolThreads = 256;
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) meanpool_kernel(const bf16* __restrict__ x,
                                                                 int N, int nB, HeadList items,
-                                                                float* __restrict__ out) {
+                                                                double* __restrict__ out) {
     constexpr int kCPR = D / 8;          // 16-byte chunks per row
     constexpr int kGroups = 32 / kCPR;   // row groups per warp
     constexpr int kRows = 64 / kGroups;  // rows per lane
@@ -56,12 +56,10 @@ __global__ void __launch_bounds__(kPoolThreads) meanpool_kernel(const bf16* __re
     for (int off = kCPR; off < 32; off <<= 1)
 #pragma unroll
         for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], off);
-    if (grp == 0) {
-        float4* o = reinterpret_cast<float4*>(out + ((size_t)item * nB + b) * D + c * 8);
-        o[0] = make_float4((float)(acc[0] / 64.0), (float)(acc[1] / 64.0), (float)(acc[2] / 64.0),
-                           (float)(acc[3] / 64.0));
-        o[1] = make_float4((float)(acc[4] / 64.0), (float)(acc[5] / 64.0), (float)(acc[6] / 64.0),
-                           (float)(acc[7] / 64.0));
+    if (grp == 0) {  // the means, exact in fp64 (a power-of-two division)
+        double2* o = reinterpret_cast<double2*>(out + ((size_t)item * nB + b) * D + c * 8);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) o[v] = make_double2(acc[2 * v] / 64.0, acc[2 * v + 1] / 64.0);
     }
 }
 
@@ -109,7 +107,7 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 //          its row of S, ties toward the lower block, output ascending.
 template <int D>
 __global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
-    const float* __restrict__ qm, const float* __restrict__ km, int Hq, int Hkv, int nB,
+    const double* __restrict__ qm, const double* __restrict__ km, int Hq, int Hkv, int nB,
     int kvmap_n, HeadList heads, HeadList kvpos, int R, double scale, int topk, RowCounts tk,
     int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt) {
     constexpr int RS = bs_row<D>();
@@ -129,47 +127,39 @@ __global__ void __launch_bounds__(kTopkThreads, 1) bs_topk_kernel(
     int gi = 0;
     for (int t = 0; t < kvmap_n; ++t)
         if (head_qh(kvpos.e[t]) == g) gi = t;
-    const float* kmg = km + (size_t)gi * nB * D;
+    const double* kmg = km + (size_t)gi * nB * D;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    // rows widened to fp64 once; rows past nr read 0
-    for (int t = threadIdx.x; t < kMaxR * (D / 4); t += blockDim.x) {
-        const int r = t / (D / 4), c4 = t % (D / 4);
-        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nr) f = *reinterpret_cast<const float4*>(qm + ((size_t)pos * nB + bq0 + r) * D + 4 * c4);
-        double* d = Qs + r * RS + 4 * c4;
-        d[0] = f.x;
-        d[1] = f.y;
-        d[2] = f.z;
-        d[3] = f.w;
+    // the rows' means; rows past nr read 0
+    for (int t = threadIdx.x; t < kMaxR * (D / 2); t += blockDim.x) {
+        const int r = t / (D / 2), c2 = t % (D / 2);
+        double2 f = make_double2(0.0, 0.0);
+        if (r < nr) f = *reinterpret_cast<const double2*>(qm + ((size_t)pos * nB + bq0 + r) * D + 2 * c2);
+        *reinterpret_cast<double2*>(Qs + r * RS + 2 * c2) = f;
     }
     const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
     // the key tile is fetched one tile ahead into registers, so that its global
     // loads are in flight while the MMAs of the current tile run
-    constexpr int kPf = kKeyTile * (D / 4) / kTopkThreads;  // float4 per thread per tile
-    float4 pf[kPf];
+    constexpr int kPf = kKeyTile * (D / 2) / kTopkThreads;  // double2 per thread per tile
+    double2 pf[kPf];
     auto fetch = [&](int kt) {
 #pragma unroll
         for (int u = 0; u < kPf; ++u) {
             const int t = threadIdx.x + u * kTopkThreads;
-            const int kb = t / (D / 4), c4 = t % (D / 4);
-            pf[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int kb = t / (D / 2), c2 = t % (D / 2);
+            pf[u] = make_double2(0.0, 0.0);
             if (kt + kb < ncand)
-                pf[u] = *reinterpret_cast<const float4*>(kmg + (size_t)(kt + kb) * D + 4 * c4);
+                pf[u] = *reinterpret_cast<const double2*>(kmg + (size_t)(kt + kb) * D + 2 * c2);
         }
     };
     fetch(0);
     for (int kt0 = 0; kt0 < ncand; kt0 += kKeyTile) {
         __syncthreads();  // the previous tile has been used
 #pragma unroll
-        for (int u = 0; u < kPf; ++u) {
+        for (int u = 0; u < kPf; ++u) {  // consecutive lanes, consecutive 16 bytes
             const int t = threadIdx.x + u * kTopkThreads;
-            const int kb = t / (D / 4), c4 = t % (D / 4);
-            double* d = Ks + kb * RS + 4 * c4;
-            d[0] = pf[u].x;
-            d[1] = pf[u].y;
-            d[2] = pf[u].z;
-            d[3] = pf[u].w;
+            const int kb = t / (D / 2), c2 = t % (D / 2);
+            *reinterpret_cast<double2*>(Ks + kb * RS + 2 * c2) = pf[u];
         }
         __syncthreads();
         if (kt0 + kKeyTile < ncand) fetch(kt0 + kKeyTile);
@@ -255,8 +245,8 @@ cudaError_t launch_bs_d(const bf16* q, const bf16* k, int Hq, int Hkv, int N, do
 BsIndexWs carve_bs_index(WsCarver& c, int n_heads, int Hkv, int N, int d) {
     BsIndexWs w{};
     const int nB = N / 64;
-    w.qm = c.take<float>((size_t)n_heads * nB * d);
-    w.km = c.take<float>((size_t)Hkv * nB * d);
+    w.qm = c.take<double>((size_t)n_heads * nB * d);
+    w.km = c.take<double>((size_t)Hkv * nB * d);
     return w;
 }
 

@@ -90,8 +90,8 @@ cudaError_t read_vs_wait_failure(int* out8);
 
 // ----------------------------------------------------------- BS index
 struct BsIndexWs {
-    float* qm;  // [n_heads][nB][d]
-    float* km;  // [Hkv][nB][d]
+    double* qm;  // [n_heads][nB][d] block means
+    double* km;  // [Hkv][nB][d]
 };
 BsIndexWs carve_bs_index(WsCarver& c, int n_heads, int Hkv, int N, int d);
 // topk: budget and index row stride; topk_rows (optional, host, one per listed

@@ -153,7 +153,7 @@ int mi_vs_index(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int 
  * "Block-Sparse Kernel Mechanics": block score against the mean key of each
  * block, keep the top-k).  Qm[b] / Km[b] are means of 64 rows; for query
  * block bq the candidates are key blocks bk <= bq with score
- * scale * Qm[bq] . Km[bk] (fp64 sums of fp32 means).  The top
+ * scale * Qm[bq] . Km[bk] (fp64 means and fp64 dot products).  The top
  * min(topk, bq+1) (ties: lower block first) are written sorted ascending:
  *   blk_idx [n_heads][N/64][topk] int32 (device; unused entries -1),
  *   blk_cnt [n_heads][N/64] int32 (device).
