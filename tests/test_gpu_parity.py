@@ -31,10 +31,10 @@ def _built():
 @pytest.mark.parametrize("Hq,Hkv,N,d,L,kv,ks", [
     (1, 1, 2048, 64, 64, 128, 256),     # the 2K single-head workload
     (4, 1, 1088, 128, 64, 100, 300),    # GQA 4:1, ragged N
-    (2, 2, 640, 128, 130, 700, 17),     # last_q not a multiple of 64, kv > N (clamped)
+    (2, 2, 640, 128, 130, 700, 17),     # last_q not a multiple of 64 (3 row groups), kv > N
     (2, 1, 192, 64, 64, 0, 1),          # tiny: one super tile, zero vertical budget
-    # tensor-core score passes (last_q <= 64): several 2048-key chunks, so diagonals
-    # that start near a chunk's end are finished in the next key tile, plus ragged tails
+    # several 2048-key chunks, so diagonals that start near a chunk's end are finished
+    # in the next key tile, plus ragged tails
     (2, 1, 4160, 128, 64, 300, 900),    # 3 chunks, the last one 64 keys
     (3, 1, 6144, 64, 48, 200, 500),     # 3 full chunks, 16 padding rows per head, odd head count
     (1, 1, 4096, 128, 1, 100, 300),     # last_q = 1: a single row, diagonals of one element
@@ -252,13 +252,14 @@ def test_full_budgets_equal_dense_sdpa():
         assert err.max().item() <= 1e-2 and err.mean().item() <= 1e-3
 
 
-@pytest.mark.parametrize("N,d", [(1024, 128), (576, 64)])
-def test_prefill_layer_mixed_matches_oracle(N, d):
-    """The pattern router: mixed A-shape / VS / BS / dense heads in one launch."""
+@pytest.mark.parametrize("N,d,L", [(1024, 128, 64), (576, 64, 64), (2560, 128, 100)])
+def test_prefill_layer_mixed_matches_oracle(N, d, L):
+    """The pattern router: mixed A-shape / VS / BS / dense heads in one launch
+    (last_q = 100: the VS index merges two 64-row groups per head)."""
     w = synth.workload("mixed_n256k_llama3_8b", Hq=8, Hkv=2, N=N, d=d)
     x = synth.make_inputs(w, device="cuda")
     pattern = np.array([0, 1, 2, 3, 2, 0, 1, 3], np.int8)
-    p = B.make_params(last_q=64, vertical_size=40, slash_size=60, topk_blocks=4, sink=64,
+    p = B.make_params(last_q=L, vertical_size=40, slash_size=60, topk_blocks=4, sink=64,
                       window=256)
     out, lse = B.mi_prefill_layer(x["q"], x["k"], x["v"], pattern, p, want_lse=True)
     torch.cuda.synchronize()
@@ -267,7 +268,7 @@ def test_prefill_layer_mixed_matches_oracle(N, d):
         if pattern[h] == 0:
             ro, rl = oracle.attn_ashape(qs, ks_, vs_, 0, 64, 256)
         elif pattern[h] == 1:
-            a, b, _, _ = oracle.vs_index(qs, ks_, 0, 64, 40, 60)
+            a, b, _, _ = oracle.vs_index(qs, ks_, 0, L, 40, 60)
             ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, a, b)
         elif pattern[h] == 3:
             ro, rl = oracle.attn_dense(qs, ks_, vs_, 0)
