@@ -165,6 +165,20 @@ def test_workspace_queries(lib):
     assert full >= vs_only > a_only >= 0
 
 
+def test_vs_index_workspace_grows_with_row_groups(lib):
+    """last_q > 64 splits each head's rows into 64-row groups whose partial
+    column and diagonal scores (fp32 [heads][groups][N], two lists) live in the
+    workspace until they are merged; last_q <= 64 needs none of them."""
+    n, N = 32, 131072
+    w64 = B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, N, 128, n, 64, 1000, 6096)
+    w1 = B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, N, 128, n, 1, 1000, 6096)
+    w200 = B.mi_workspace_bytes(B.MI_OP_VS_INDEX, 32, 8, N, 128, n, 200, 1000, 6096)
+    row_stats = lambda L: 2 * n * L * (N // 2048) * 8 + 2 * n * L * 8
+    assert w64 - w1 >= row_stats(64) - row_stats(1)
+    groups = (200 + 63) // 64
+    assert w200 - w64 >= 2 * n * groups * N * 4 + row_stats(200) - row_stats(64)
+
+
 def test_vs_index_static_validation_and_capacity(lib):
     """The no-workspace entry point validates like mi_vs_index and rejects
     shapes whose scratch exceeds its fixed array -- both before any CUDA call."""
