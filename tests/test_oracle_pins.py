@@ -321,3 +321,89 @@ def test_generator_deterministic_and_planted():
     m = synth.workload("mixed_n256k_llama3_8b")
     pt = synth.pattern_table(m, torch.Generator().manual_seed(1))
     assert sorted(np.bincount(pt, minlength=3).tolist()) == [10, 11, 11]
+
+
+# ------------------------------------------- hand-worked fixtures (golden/)
+
+def _golden_cases(name):
+    """Blank-line separated `key: value` blocks of a hand-worked fixture file."""
+    cases, cur = [], {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].rstrip()
+            if not line:
+                if cur:
+                    cases.append(cur)
+                    cur = {}
+                continue
+            key, _, val = line.partition(":")
+            cur[key.strip()] = val.strip()
+    if cur:
+        cases.append(cur)
+    return [pytest.param(c, id=c.get("case")) for c in cases]
+
+
+def _fracs(s):
+    from fractions import Fraction
+    return np.array([float(Fraction(t)) for t in s.split()], np.float64)
+
+
+def _rows(s):
+    """'a b | c d ; e f | g h' -> float32 [heads, rows, cols]."""
+    heads = [[[float(x) for x in r.split()] for r in h.split("|")] for h in s.split(";")]
+    return torch.tensor(heads, dtype=torch.float32)
+
+
+def _ints(s):
+    return [int(t) for t in s.split()]
+
+
+@pytest.mark.parametrize("c", _golden_cases("vs_scores_hand.txt"))
+def test_vs_scores_hand_worked(c):
+    """Column and diagonal sums equal fractions worked by hand (weights 2^(q.k))."""
+    q, k = _rows(c["q"]), _rows(c["k"])
+    h, L = int(c["h"]), int(c["last_q"])
+    assert q.shape == (int(c["Hq"]), int(c["N"]), int(c["d"])) and k.shape[0] == int(c["Hkv"])
+    vert, sl = oracle.vs_scores(q, k, h, L, scale=np.log(2.0))
+    np.testing.assert_allclose(vert, _fracs(c["vertical"]), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(sl, _fracs(c["slash"]), rtol=1e-14, atol=1e-15)
+    for kk in (1, 2):
+        assert oracle.topk(vert, kk).tolist() == _ints(c[f"v_top{kk}"])
+        assert oracle.topk(sl, kk).tolist() == _ints(c[f"s_top{kk}"])
+
+
+@pytest.mark.parametrize("c", _golden_cases("bs_index_hand.txt"))
+def test_bs_index_hand_worked(c):
+    """Block means, causal block scores and top-k equal values worked by hand."""
+    N, d, B = int(c["N"]), int(c["d"]), int(c["block"])
+    q, k = _rows(c["q"]), _rows(c["k"])
+    assert q.shape == (1, N, d) and k.shape == (1, N, d)
+    nB = N // B
+    want_s = [[float(x) for x in r.split()] for r in c["scores"].split(";")]
+    for kk in (1, 2):
+        bi, bc, sc = oracle.bs_index(q, k, 0, kk, block=B, scale=1.0, want_scores=True)
+        want = [_ints(r) for r in c[f"top{kk}"].split(";")]
+        for bq in range(nB):
+            np.testing.assert_allclose(sc[bq, :bq + 1], want_s[bq], rtol=0, atol=1e-15)
+            assert bc[bq] == len(want[bq]) and bi[bq, :bc[bq]].tolist() == want[bq]
+
+
+@pytest.mark.parametrize("c", _golden_cases("attn_hand.txt"))
+def test_attention_hand_worked(c):
+    """A-shape and Vertical-Slash rows (window, gathered column, no double count,
+    empty rows) equal fractions worked by hand."""
+    N = int(c["N"])
+    q = torch.ones(1, N, 1)
+    k = torch.tensor(_ints(c["k"]), dtype=torch.float32).reshape(1, N, 1)
+    v = torch.tensor(_ints(c["v"]), dtype=torch.float32).reshape(1, N, 1)
+    if c["case"] == "ashape":
+        out, lse = oracle.attn_ashape(q, k, v, 0, int(c["sink"]), int(c["window"]),
+                                      scale=np.log(2.0))
+    else:
+        out, lse = oracle.attn_vs(q, k, v, 0, _ints(c["v_idx"]), _ints(c["s_idx"]),
+                                  block=int(c["block"]), scale=np.log(2.0))
+    np.testing.assert_allclose(out[:, 0], _fracs(c["out"]), rtol=1e-14, atol=1e-15)
+    lse_of = _fracs(c["lse_of"])
+    empty = lse_of == 0
+    assert np.all(np.isneginf(lse[empty]))
+    np.testing.assert_allclose(lse[~empty], np.log(lse_of[~empty]), rtol=1e-14, atol=1e-15)
