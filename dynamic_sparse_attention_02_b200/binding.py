@@ -120,17 +120,62 @@ def _check(fn, rc):
         raise MinferError(fn, rc)
 
 
-def _shape(q, k):
+def _dev(name, t, dtype, shape, device):
+    """The library reads raw device pointers with the layout the header states:
+    refuse anything else before a pointer reaches a kernel (a host pointer, a
+    wrong element type or a strided view would be read as dense device data)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not _device_ok(t, device):
+        raise ValueError(f"{name} must be on {device or 'a CUDA device'}, got {t.device}")
+
+
+def _device_ok(t, device):
+    return t.device.type == "cuda" and (device is None or t.device == device)
+
+
+def _shape(q, k, v=None):
+    """(Hq, Hkv, N, d) of bf16 [Hq, N, d] q and [Hkv, N, d] k (and v) on one device."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise ValueError("q must be a 3-D tensor [Hq, N, d]")
     Hq, N, d = q.shape
-    return Hq, k.shape[0], N, d
+    _dev("q", q, torch.bfloat16, None, None)
+    if not isinstance(k, torch.Tensor) or k.dim() != 3:
+        raise ValueError("k must be a 3-D tensor [Hkv, N, d]")
+    Hkv = k.shape[0]
+    _dev("k", k, torch.bfloat16, (Hkv, N, d), q.device)
+    _dev("v", v, torch.bfloat16, (Hkv, N, d), q.device)
+    return Hq, Hkv, N, d
+
+
+def _host_array(name, a, dtype, n):
+    arr = np.ascontiguousarray(np.asarray(a, dtype=dtype))
+    if arr.ndim != 1 or arr.size != n:
+        raise ValueError(f"{name} must hold {n} entries, got shape {arr.shape}")
+    return arr
 
 
 def _workspace(nbytes, device, ws):
+    """(tensor, its size in bytes): the caller's workspace, checked, or a new one."""
     if ws is not None:
-        if ws.numel() * ws.element_size() < nbytes:
-            raise ValueError("workspace too small")
-        return ws
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        if not isinstance(ws, torch.Tensor) or not ws.is_contiguous():
+            raise ValueError("ws must be a contiguous tensor")
+        if not _device_ok(ws, device):
+            raise ValueError(f"ws must be on {device}, got {ws.device}")
+        size = ws.numel() * ws.element_size()
+        if size < nbytes:
+            raise ValueError(f"workspace too small: {size} < {nbytes} bytes")
+        return ws, size
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    return ws, ws.numel()
 
 
 def mi_debug_wait_failure():
@@ -161,22 +206,33 @@ def make_params(last_q=64, vertical_size=1000, slash_size=6096, topk_blocks=100,
 
 
 def mi_prefill_workspace_bytes(Hq, Hkv, N, d, pattern, params: mi_params) -> int:
-    pat = None if pattern is None else np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
+    pat = None if pattern is None else _host_array("pattern", pattern, np.int8, Hq)
     pp = None if pat is None else pat.ctypes.data_as(ctypes.c_void_p)
     return int(_lib_handle().mi_prefill_workspace_bytes(Hq, Hkv, N, d, pp, ctypes.byref(params)))
 
 
-def _params_array(params):
-    arr = (mi_params * len(params))(*params)
-    return arr
+def _params_array(params, Hq):
+    if len(params) != Hq:
+        raise ValueError(f"one mi_params per query head: {Hq} expected, got {len(params)}")
+    return (mi_params * Hq)(*params)
 
 
 def mi_prefill_workspace_bytes_heads(Hq, Hkv, N, d, pattern, params) -> int:
     """Workspace of mi_prefill_layer_heads: `params` holds one mi_params per head."""
-    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
-    arr = _params_array(params)
+    pat = _host_array("pattern", pattern, np.int8, Hq)
+    arr = _params_array(params, Hq)
     return int(_lib_handle().mi_prefill_workspace_bytes_heads(
         Hq, Hkv, N, d, pat.ctypes.data_as(ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p)))
+
+
+def _index_outputs(n, N, vertical_size, slash_size, want_scores, dev):
+    if vertical_size < 0 or slash_size < 0:
+        raise ValueError("budgets must be non-negative")
+    v_idx = torch.empty(n, vertical_size, dtype=torch.int32, device=dev)
+    s_idx = torch.empty(n, slash_size, dtype=torch.int32, device=dev)
+    vs = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    ss = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    return v_idx, s_idx, vs, ss
 
 
 def mi_vs_index(q, k, last_q, vertical_size, slash_size, heads: Optional[Sequence[int]] = None,
@@ -185,15 +241,12 @@ def mi_vs_index(q, k, last_q, vertical_size, slash_size, heads: Optional[Sequenc
     Hq, Hkv, N, d = _shape(q, k)
     harr, n, hp = _heads(heads, Hq)
     dev = q.device
-    v_idx = torch.empty(n, vertical_size, dtype=torch.int32, device=dev)
-    s_idx = torch.empty(n, slash_size, dtype=torch.int32, device=dev)
-    vs = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
-    ss = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    v_idx, s_idx, vs, ss = _index_outputs(n, N, vertical_size, slash_size, want_scores, dev)
     nb = mi_workspace_bytes(MI_OP_VS_INDEX, Hq, Hkv, N, d, n, last_q, vertical_size, slash_size)
-    ws = _workspace(nb, dev, ws)
+    ws, ws_bytes = _workspace(nb, dev, ws)
     rc = _lib_handle().mi_vs_index(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, last_q, vertical_size,
                                    slash_size, hp, n, _ptr(v_idx), _ptr(s_idx), _ptr(vs), _ptr(ss),
-                                   _ptr(ws), ws.numel(), _stream(stream))
+                                   _ptr(ws), ws_bytes, _stream(stream))
     _check("mi_vs_index", rc)
     return (v_idx, s_idx, vs, ss) if want_scores else (v_idx, s_idx)
 
@@ -204,11 +257,7 @@ def mi_vs_index_static(q, k, last_q, vertical_size, slash_size, heads=None, scal
     the scratch in a fixed 16 MiB device array (calls must not overlap)."""
     Hq, Hkv, N, d = _shape(q, k)
     harr, n, hp = _heads(heads, Hq)
-    dev = q.device
-    v_idx = torch.empty(n, vertical_size, dtype=torch.int32, device=dev)
-    s_idx = torch.empty(n, slash_size, dtype=torch.int32, device=dev)
-    vs = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
-    ss = torch.empty(n, N, dtype=torch.float32, device=dev) if want_scores else None
+    v_idx, s_idx, vs, ss = _index_outputs(n, N, vertical_size, slash_size, want_scores, q.device)
     rc = _lib_handle().mi_vs_index_static(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, last_q,
                                           vertical_size, slash_size, hp, n, _ptr(v_idx),
                                           _ptr(s_idx), _ptr(vs), _ptr(ss), _stream(stream))
@@ -220,37 +269,57 @@ def mi_bs_index(q, k, topk, heads=None, scale=0.0, ws=None, stream=None):
     """Block-Sparse index: (blk_idx [n, N/64, topk], blk_cnt [n, N/64])."""
     Hq, Hkv, N, d = _shape(q, k)
     harr, n, hp = _heads(heads, Hq)
+    if topk < 0:
+        raise ValueError("topk must be non-negative")
     dev = q.device
     nB = N // MI_BLOCK
     blk_idx = torch.empty(n, nB, topk, dtype=torch.int32, device=dev)
     blk_cnt = torch.empty(n, nB, dtype=torch.int32, device=dev)
-    ws = _workspace(mi_workspace_bytes(MI_OP_BS_INDEX, Hq, Hkv, N, d, n), dev, ws)
+    ws, ws_bytes = _workspace(mi_workspace_bytes(MI_OP_BS_INDEX, Hq, Hkv, N, d, n), dev, ws)
     rc = _lib_handle().mi_bs_index(_ptr(q), _ptr(k), Hq, Hkv, N, d, scale, MI_BLOCK, topk, hp, n,
-                                   _ptr(blk_idx), _ptr(blk_cnt), _ptr(ws), ws.numel(),
+                                   _ptr(blk_idx), _ptr(blk_cnt), _ptr(ws), ws_bytes,
                                    _stream(stream))
     _check("mi_bs_index", rc)
     return blk_idx, blk_cnt
 
 
-def _attn_out(q, out, lse, want_lse):
+def _attn_out(q, out, lse, want_lse, err_count):
+    """Check or allocate out (bf16 [Hq, N, d]) and lse (fp32 [Hq, N]); check err_count."""
+    Hq, N, _ = q.shape
+    _dev("out", out, torch.bfloat16, q.shape, q.device)
+    _dev("lse", lse, torch.float32, (Hq, N), q.device)
+    _dev("err_count", err_count, torch.int32, None, q.device)
+    if err_count is not None and err_count.numel() < 1:
+        raise ValueError("err_count must hold one int32")
     if out is None:
         out = torch.zeros_like(q)
     if lse is None and want_lse:
-        lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device=q.device)
+        lse = torch.full((Hq, N), float("nan"), dtype=torch.float32, device=q.device)
     return out, lse
+
+
+def _index_rows(name, t, n, q):
+    """An int32 index tensor with one row per listed head; returns its row length."""
+    if t is None:
+        return 0
+    if not isinstance(t, torch.Tensor) or t.dim() != 2 or t.shape[0] != n:
+        raise ValueError(f"{name} must be a 2-D int32 tensor with {n} rows")
+    _dev(name, t, torch.int32, None, q.device)
+    return int(t.shape[1])
 
 
 def mi_vs_sparse_attn(q, k, v, v_idx, s_idx, heads=None, scale=0.0, out=None, lse=None,
                       want_lse=True, err_count=None, ws=None, stream=None):
-    Hq, Hkv, N, d = _shape(q, k)
+    Hq, Hkv, N, d = _shape(q, k, v)
     harr, n, hp = _heads(heads, Hq)
-    out, lse = _attn_out(q, out, lse, want_lse)
-    kv = v_idx.shape[-1] if v_idx is not None else 0
-    ks = s_idx.shape[-1] if s_idx is not None else 0
-    ws = _workspace(mi_workspace_bytes(MI_OP_VS_ATTN, Hq, Hkv, N, d, n, 0, kv, ks), q.device, ws)
+    kv = _index_rows("v_idx", v_idx, n, q)
+    ks = _index_rows("s_idx", s_idx, n, q)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
+    ws, ws_bytes = _workspace(mi_workspace_bytes(MI_OP_VS_ATTN, Hq, Hkv, N, d, n, 0, kv, ks),
+                              q.device, ws)
     rc = _lib_handle().mi_vs_sparse_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
                                          _ptr(v_idx), kv, _ptr(s_idx), ks, hp, n, _ptr(out),
-                                         _ptr(lse), _ptr(err_count), _ptr(ws), ws.numel(),
+                                         _ptr(lse), _ptr(err_count), _ptr(ws), ws_bytes,
                                          _stream(stream))
     _check("mi_vs_sparse_attn", rc)
     return out, lse
@@ -258,10 +327,15 @@ def mi_vs_sparse_attn(q, k, v, v_idx, s_idx, heads=None, scale=0.0, out=None, ls
 
 def mi_block_sparse_attn(q, k, v, blk_idx, blk_cnt, heads=None, scale=0.0, out=None, lse=None,
                          want_lse=True, err_count=None, stream=None):
-    Hq, Hkv, N, d = _shape(q, k)
+    Hq, Hkv, N, d = _shape(q, k, v)
     harr, n, hp = _heads(heads, Hq)
-    out, lse = _attn_out(q, out, lse, want_lse)
-    topk = blk_idx.shape[-1]
+    nB = N // MI_BLOCK
+    if not isinstance(blk_idx, torch.Tensor) or blk_idx.dim() != 3:
+        raise ValueError("blk_idx must be a 3-D int32 tensor [n_heads, N/64, topk]")
+    topk = int(blk_idx.shape[-1])
+    _dev("blk_idx", blk_idx, torch.int32, (n, nB, topk), q.device)
+    _dev("blk_cnt", blk_cnt, torch.int32, (n, nB), q.device)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
     rc = _lib_handle().mi_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
                                             _ptr(blk_idx), _ptr(blk_cnt), topk, MI_BLOCK, hp, n,
                                             _ptr(out), _ptr(lse), _ptr(err_count), None, 0,
@@ -272,9 +346,9 @@ def mi_block_sparse_attn(q, k, v, blk_idx, blk_cnt, heads=None, scale=0.0, out=N
 
 def mi_ashape_attn(q, k, v, sink, window, heads=None, scale=0.0, out=None, lse=None,
                    want_lse=True, err_count=None, stream=None):
-    Hq, Hkv, N, d = _shape(q, k)
+    Hq, Hkv, N, d = _shape(q, k, v)
     harr, n, hp = _heads(heads, Hq)
-    out, lse = _attn_out(q, out, lse, want_lse)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
     rc = _lib_handle().mi_ashape_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, sink,
                                       window, hp, n, _ptr(out), _ptr(lse), _ptr(err_count), None,
                                       0, _stream(stream))
@@ -285,9 +359,9 @@ def mi_ashape_attn(q, k, v, sink, window, heads=None, scale=0.0, out=None, lse=N
 def mi_dense_attn(q, k, v, heads=None, scale=0.0, out=None, lse=None, want_lse=True,
                   err_count=None, stream=None):
     """Dense causal attention (every key j <= i) on the same engine."""
-    Hq, Hkv, N, d = _shape(q, k)
+    Hq, Hkv, N, d = _shape(q, k, v)
     harr, n, hp = _heads(heads, Hq)
-    out, lse = _attn_out(q, out, lse, want_lse)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
     rc = _lib_handle().mi_dense_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, hp, n,
                                      _ptr(out), _ptr(lse), _ptr(err_count), None, 0,
                                      _stream(stream))
@@ -298,18 +372,16 @@ def mi_dense_attn(q, k, v, heads=None, scale=0.0, out=None, lse=None, want_lse=T
 def mi_prefill_layer_heads(q, k, v, pattern, params, scale=0.0, out=None, lse=None,
                            want_lse=False, err_count=None, ws=None, stream=None):
     """One layer with one mi_params per head (host int8 pattern [Hq], params [Hq])."""
-    Hq, Hkv, N, d = _shape(q, k)
-    if len(params) != Hq:
-        raise ValueError("one mi_params per query head")
-    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
-    arr = _params_array(params)
-    out, lse = _attn_out(q, out, lse, want_lse)
+    Hq, Hkv, N, d = _shape(q, k, v)
+    pat = _host_array("pattern", pattern, np.int8, Hq)
+    arr = _params_array(params, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
     need = mi_prefill_workspace_bytes_heads(Hq, Hkv, N, d, pat, params)
-    ws = _workspace(need, q.device, ws)
+    ws, ws_bytes = _workspace(need, q.device, ws)
     rc = _lib_handle().mi_prefill_layer_heads(
         _ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, pat.ctypes.data_as(ctypes.c_void_p),
         ctypes.cast(arr, ctypes.c_void_p), _ptr(out), _ptr(lse), _ptr(err_count), _ptr(ws),
-        ws.numel(), _stream(stream), None)
+        ws_bytes, _stream(stream), None)
     _check("mi_prefill_layer_heads", rc)
     return out, lse
 
@@ -317,12 +389,15 @@ def mi_prefill_layer_heads(q, k, v, pattern, params, scale=0.0, out=None, lse=No
 def mi_prefill_layer(q, k, v, pattern, params: mi_params, scale=0.0, out=None, lse=None,
                      want_lse=False, err_count=None, ws=None, stage_events=None, stream=None):
     """One layer: per-head pattern table (host int8 [Hq]) -> index + sparse attention."""
-    Hq, Hkv, N, d = _shape(q, k)
-    pat = np.ascontiguousarray(np.asarray(pattern, dtype=np.int8))
-    out, lse = _attn_out(q, out, lse, want_lse)
-    ws = _workspace(mi_prefill_workspace_bytes(Hq, Hkv, N, d, pat, params), q.device, ws)
+    Hq, Hkv, N, d = _shape(q, k, v)
+    pat = _host_array("pattern", pattern, np.int8, Hq)
+    out, lse = _attn_out(q, out, lse, want_lse, err_count)
+    ws, ws_bytes = _workspace(mi_prefill_workspace_bytes(Hq, Hkv, N, d, pat, params), q.device,
+                              ws)
     ev = None
     if stage_events is not None:
+        if len(stage_events) != MI_STAGE_EVENTS:
+            raise ValueError(f"stage_events must hold {MI_STAGE_EVENTS} events")
         for e in stage_events:
             if not e.cuda_event:  # torch creates the CUDA event on first record
                 e.record()
@@ -330,6 +405,6 @@ def mi_prefill_layer(q, k, v, pattern, params: mi_params, scale=0.0, out=None, l
     rc = _lib_handle().mi_prefill_layer(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
                                         pat.ctypes.data_as(ctypes.c_void_p), ctypes.byref(params),
                                         _ptr(out), _ptr(lse), _ptr(err_count), _ptr(ws),
-                                        ws.numel(), _stream(stream), ev)
+                                        ws_bytes, _stream(stream), ev)
     _check("mi_prefill_layer", rc)
     return out, lse
