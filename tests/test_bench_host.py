@@ -40,3 +40,27 @@ def test_ashape_tile_count_matches_brute_force():
         b = np.arange(nB)[None, :]
         want = int(np.sum((b <= qb) & ((64 * b < sink) | (64 * (qb - b) - 63 < window))))
         assert bench.ashape_tiles(N, sink, window) == want
+
+
+def test_clock_samples_summary():
+    """Median SM clock, highest max clock, and every slowdown reason seen Active;
+    unreadable fields and short lines are skipped."""
+    idle = "Not Active"
+    lines = [
+        f"0, 1700, 1965, 900.1, 0x4, {idle}, {idle}, {idle}, Active\n",
+        f"0, 1650, 1965, 990.0, 0x4, {idle}, {idle}, {idle}, Active\n",
+        f"0, 1800, 1965, 700.0, 0x0, {idle}, {idle}, {idle}, {idle}\n",
+        f"0, [N/A], 1965, 700.0, 0x0, {idle}, Active, {idle}, {idle}\n",
+        "garbage line\n",
+    ]
+    got = bench.parse_clock_samples(lines)
+    assert got["sm_mhz"] == 1700.0 and got["sm_max_mhz"] == 1965.0
+    assert got["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert got["samples"] == 4
+    assert bench.parse_clock_samples([])["reasons"] == ["no samples"]
+
+
+def test_job_value_is_whole_job_time_per_layer():
+    """N replicas each finish one layer per step, timed by the slowest rank."""
+    assert bench.job_value(130.0, 1) == 130.0
+    assert bench.job_value(132.0, 4) == 33.0
