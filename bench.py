@@ -281,7 +281,7 @@ def config_of(w):
 class Ranks:
     """One process per GPU, launched by torchrun: rank and world size from its
     environment, and a process group for the barriers around the timed region
-    and the max-over-ranks step time (NCCL on the GPU machine; the tests drive the
+    and the max-over-ranks step time (NCCL on GPUs; the tests drive the
     same code over gloo on CPU).  The layer is run as independent replicas:
     no collective touches the data path."""
 
