@@ -64,3 +64,31 @@ def test_job_value_is_whole_job_time_per_layer():
     """N replicas each finish one layer per step, timed by the slowest rank."""
     assert bench.job_value(130.0, 1) == 130.0
     assert bench.job_value(132.0, 4) == 33.0
+
+
+def test_reference_arm_json_line(capsys, monkeypatch):
+    """`--impl reference` prints one JSON line with the contract's keys: the
+    oracle timed on a bounded sample, host-only (no copies), time-like metric."""
+    import json
+    for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(key, raising=False)
+    args = bench.parse_args(["--impl", "reference", "--steps", "2", "--warmup", "3",
+                             "--workload", "vs_n2k_h1_d64"])
+    assert bench.run_reference(args) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["n_gpus"] == 1
+    assert (d["steps"], d["warmup"]) == (2, 3)
+    assert d["higher_is_better"] is False and d["vs_baseline"] is None
+    assert d["value"] > 0 and d["ms_per_step"] == d["value"]
+    assert d["config"]["workload"] == "vs_n2k_h1_d64" and d["config"]["N"] == 2048
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert "2048 seeded random rows" in cb["sample"]  # the whole small layer was sampled
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
