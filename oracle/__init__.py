@@ -20,6 +20,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "minfer_oracle.c")
 _LIB = os.path.join(_HERE, "libminfer_oracle.so")
+# A prebuilt variant of the oracle to load instead (the mutation test plants
+# mistakes in copies of minfer_oracle.c and runs the pins against each).
+_VARIANT = os.environ.get("MINFER_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -38,7 +41,7 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            lib = ctypes.CDLL(_VARIANT or build())
             P = ctypes.c_void_p
             I, I64, D = ctypes.c_int, ctypes.c_int64, ctypes.c_double
             lib.oracle_vs_scores.argtypes = [P, P, I, I, I, I, D, I, I, P, P]

@@ -153,7 +153,7 @@ def test_vs_mask_matches_brute_force():
     Hq, Hkv, N, d = 2, 1, 512, 64
     q, k, v = rand_qkv(Hq, Hkv, N, d, 9)
     v_idx = np.array([3, 77, 200, 201, 450], np.int32)
-    s_idx = np.array([0, 100, 300], np.int32)
+    s_idx = np.array([0, 100, 300, 385], np.int32)  # 385 = 6*64 + 1 touches deltas 6 and 7
     D = set()
     for o in s_idx:  # tiles touched by each diagonal, by scanning its elements
         for i in range(N):
@@ -197,6 +197,11 @@ def test_slash_deltas_brute_force_scan():
                 want.add(i // 64 - (i - o) // 64)
         D = oracle.slash_deltas(offs, N)
         assert set(np.nonzero(D)[0].tolist()) == want
+    # each offset alone at and beside a block boundary, where a bound is easiest to get wrong
+    for o in [64 * a + r for a in (0, 1, 7, 15) for r in (0, 1, 2, 62, 63)]:
+        want = {i // 64 - (i - o) // 64 for i in range(o, N)}
+        D = oracle.slash_deltas(np.array([o], np.int32), N)
+        assert set(np.nonzero(D)[0].tolist()) == want, o
 
 
 def _softmax_weights_via_sdpa(q, k, h, rows):
