@@ -135,3 +135,15 @@ def test_valid_layer_call_marshals_the_tables(fake):
     args = fake.calls[-1][1]
     assert args[3:7] == (4, 2, 256, 64)
     assert args[14] == 4096
+
+
+def test_missing_library_raises_instead_of_falling_back(monkeypatch):
+    """Without the built library every entry point raises: there is no CPU path."""
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", B.LIB_PATH + ".absent")
+    monkeypatch.setattr(B, "_device_ok", lambda t, dev: dev is None or t.device == dev)
+    q, k, v = bf16(2, 128, 64), bf16(1, 128, 64), bf16(1, 128, 64)
+    with pytest.raises(RuntimeError, match="is not built"):
+        B.mi_dense_attn(q, k, v, stream=0)
+    with pytest.raises(RuntimeError, match="is not built"):
+        B.mi_prefill_layer(q, k, v, [1, 2], B.make_params(), stream=0)
