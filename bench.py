@@ -64,6 +64,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense-prefill comparison (every head dense causal)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-1m", action="store_true",
+                    help="skip the 1M-token layer measured after the main workload (at_1m)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0,
                     help="approximate CPU seconds for the oracle baseline sample")
     return ap.parse_args(argv)
@@ -104,6 +106,21 @@ def recorded_traffic(workload):
     if not entry or entry.get("source_sha") != attn_source_sha():
         return None
     return entry.get("dram_bytes_per_launch")
+
+
+def recorded_tensor_pipe(workload):
+    """Tensor-pipe utilisation of the attention kernel from a committed ncu
+    summary taken on the current kernel source (else None).  The capture is a
+    small case of the same pattern (the record says which)."""
+    path = os.path.join(ROOT, "profiles", "attn_tensor_pipe.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    entry = rec.get(workload)
+    if not entry or entry.get("source_sha") != attn_source_sha():
+        return None
+    return {k: entry[k] for k in ("pct", "metric", "case") if k in entry}
 
 
 class ClockSampler:
@@ -321,6 +338,116 @@ def job_value(ms_step_max, world):
     return ms_step_max / world
 
 
+def time_layer(B, w, x, params, ws, out, steps, warmup, ranks, dev):
+    """Warm up, then time `steps` mi_prefill_layer calls with CUDA events (stage
+    events inside each step) and nvidia-smi clock samples over the timed
+    region.  Returns (ms per step on this rank, ms index, ms prep, ms attention,
+    clock summary)."""
+    q, k, v, pattern = x["q"], x["k"], x["v"], x["pattern"]
+
+    def step(ev):
+        B.mi_prefill_layer(q, k, v, pattern, params, out=out, ws=ws, stage_events=ev)
+
+    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
+    for i in range(warmup):
+        step(warm_ev)
+        torch.cuda.synchronize()
+        log(f"{w.name} warmup step {i}: index {warm_ev[0].elapsed_time(warm_ev[1]):.2f} ms, "
+            f"attn {warm_ev[2].elapsed_time(warm_ev[3]):.2f} ms")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
+           for _ in range(steps)]
+    for e in evs:
+        for ee in e:
+            ee.record()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(steps):
+        step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    clk = clocks.stop()
+    ms_step = t_start.elapsed_time(t_end) / steps
+    ms_index = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    ms_prep = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms_attn = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    log(f"{w.name}: timed {steps} steps: {ms_step:.2f} ms/step (attn {ms_attn:.2f} ms)")
+    return ms_step, ms_index, ms_prep, ms_attn, clk
+
+
+def useful_work(B, w, x):
+    """Algorithmic work of the layer's attention launch, from its own index:
+    (computed-tile FLOPs, 64x64 tiles, gathered column-blocks)."""
+    useful, tiles, cols = 0.0, 0, 0
+    q, k, pat = x["q"], x["k"], np.asarray(x["pattern"])
+    vs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_VS]
+    bs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_BS]
+    n_ash = int(np.sum(pat == synth.PATTERN_ASHAPE))
+    if vs_heads:
+        v_idx, s_idx = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size,
+                                     heads=vs_heads)
+        vi, si = v_idx.cpu().numpy(), s_idx.cpu().numpy()
+        for i in range(len(vs_heads)):
+            f, t, c = vs_useful_flops(vi[i], si[i], w.N, w.d)
+            useful += f
+            tiles += t
+            cols += c
+    if bs_heads:
+        _, blk_cnt = B.mi_bs_index(q, k, w.topk_blocks, heads=bs_heads)
+        t = int(blk_cnt.sum().item())
+        useful += 4.0 * w.d * 64 * 64 * t
+        tiles += t
+    if n_ash:
+        t = ashape_tiles(w.N, w.sink, w.window) * n_ash
+        useful += 4.0 * w.d * 64 * 64 * t
+        tiles += t
+    return useful, tiles, cols
+
+
+def tile_density(w, tiles):
+    return tiles / (w.Hq * (w.N // 64) * (w.N // 64 + 1) / 2) if tiles else None
+
+
+def measure_1m(B, ranks, dev, peak):
+    """The metric's 1M half, measured in the same run: the 1M-token
+    Vertical-Slash layer (32 query heads, 8 KV heads, d = 128, last_q 64,
+    vertical 1000, slash 6096), 1 warm-up + 2 timed steps, with its own clock
+    record.  attn_kcycles = attention ms x median SM MHz (thousands of cycles at
+    the sampled clock), so that runs at different power-capped clocks compare."""
+    w = synth.workload("vs_n1m_llama3_8b")
+    log(f"generating {w.name} (N={w.N})")
+    x = synth.make_inputs(w, device=str(dev))
+    torch.cuda.synchronize()
+    params = params_of(w, B)
+    ws = torch.empty(B.mi_prefill_workspace_bytes(w.Hq, w.Hkv, w.N, w.d, x["pattern"], params),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x["q"])
+    steps, warmup = 2, 1
+    ms_step, ms_index, ms_prep, ms_attn, clk = time_layer(B, w, x, params, ws, out, steps,
+                                                          warmup, ranks, dev)
+    useful, tiles, cols = useful_work(B, w, x)
+    eff = useful / (ms_attn * 1e-3) / 1e12
+    mhz = clk.get("sm_mhz")
+    rec = {"workload": w.name, "N": w.N, "steps": steps, "warmup": warmup,
+           "ms_per_layer": ms_step, "ms_index": ms_index, "ms_prep": ms_prep,
+           "ms_attn": ms_attn, "eff_tflops": eff, "frac_of_peak": eff / peak,
+           "flops_per_launch": useful, "tile_density": tile_density(w, tiles),
+           "gathered_column_blocks": cols,
+           "attn_kcycles": ms_attn * mhz if mhz else None,
+           "tensor_pipe": recorded_tensor_pipe(w.name),
+           # VS index (2 score passes, row merge, top-k), prep, attention
+           "gpu_launches": 6 * steps, "clocks": clk}
+    del x, ws, out
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_minfer(args):
     from dynamic_sparse_attention_02_b200 import binding as B
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
@@ -347,40 +474,9 @@ def run_minfer(args):
     n_vs_launches = 5 + (1 if w.last_q > 64 else 0)
     launches_per_step = (n_vs_launches if n_vs else 0) + (3 if n_bs else 0) + 1
 
-    def step(ev):
-        B.mi_prefill_layer(q, k, v, pattern, params, out=out, ws=ws, stage_events=ev)
-
-    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
-    for i in range(args.warmup):
-        step(warm_ev)
-        torch.cuda.synchronize()
-        log(f"warmup step {i}: index {warm_ev[0].elapsed_time(warm_ev[1]):.2f} ms, "
-            f"attn {warm_ev[2].elapsed_time(warm_ev[3]):.2f} ms")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MI_STAGE_EVENTS)]
-           for _ in range(args.steps)]
-    for e in evs:
-        for ee in e:
-            ee.record()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index)
-    clocks.start()
-    barrier()
-    torch.cuda.synchronize()
-    t_start.record()
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record()
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms_step = t_start.elapsed_time(t_end) / args.steps
-    ms_index = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    ms_prep = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    ms_attn = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    ms_step, ms_index, ms_prep, ms_attn, clk = time_layer(B, w, x, params, ws, out, args.steps,
+                                                          args.warmup, ranks, dev)
     ms_step_max = max_over_ranks(ms_step)
-    log(f"timed {args.steps} steps: {ms_step:.2f} ms/step (attn {ms_attn:.2f} ms)")
 
     # end to end through the public API: host inputs in, host output back
     e2e = None
@@ -465,37 +561,22 @@ def run_minfer(args):
                  "tflops": 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq / (ms_dense * 1e-3) / 1e12}
         del dout
 
-    # algorithmic work of the attention launch (from this layer's own index)
-    useful = 0.0
-    tiles = 0
-    cols = 0
-    pat = np.asarray(pattern)
-    vs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_VS]
-    bs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_BS]
-    n_ash = int(np.sum(pat == synth.PATTERN_ASHAPE))
-    if vs_heads:
-        v_idx, s_idx = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size,
-                                     heads=vs_heads)
-        vi, si = v_idx.cpu().numpy(), s_idx.cpu().numpy()
-        for i in range(len(vs_heads)):
-            f, t, c = vs_useful_flops(vi[i], si[i], w.N, w.d)
-            useful += f
-            tiles += t
-            cols += c
-    if bs_heads:
-        _, blk_cnt = B.mi_bs_index(q, k, w.topk_blocks, heads=bs_heads)
-        t = int(blk_cnt.sum().item())
-        useful += 4.0 * w.d * 64 * 64 * t
-        tiles += t
-    if n_ash:
-        t = ashape_tiles(w.N, w.sink, w.window) * n_ash
-        useful += 4.0 * w.d * 64 * 64 * t
-        tiles += t
+    useful, tiles, cols = useful_work(B, w, x)
     dense_eq = 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     achieved = useful / (ms_attn * 1e-3) / 1e12 if useful else None
     traffic = recorded_traffic(w.name)
+
+    # The metric's 1M half on a single GPU (the default 128K run only).
+    at_1m = None
+    if (world == 1 and not args.no_1m and not args.seq_len
+            and w.name == "vs_n128k_llama3_8b"):
+        # the oracle baseline samples head 0 only: keep its tensors on the host
+        x = {"q": q[0:1].cpu(), "k": k[0:1].cpu(), "v": v[0:1].cpu(), "pattern": pattern}
+        del q, k, v, ws, out
+        torch.cuda.empty_cache()
+        at_1m = measure_1m(B, ranks, dev, peak)
 
     line = None
     if rank == 0:
@@ -513,7 +594,7 @@ def run_minfer(args):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config_of(w),
             "ms_index": ms_index, "ms_prep": ms_prep, "ms_attn": ms_attn,
-            "tile_density": (tiles / (w.Hq * (w.N // 64) * (w.N // 64 + 1) / 2)) if tiles else None,
+            "tile_density": tile_density(w, tiles),
             "gathered_column_blocks": cols,
             "eff_tflops": achieved,
             "dense_eq_tflops": dense_eq / (ms_step_max * 1e-3) / 1e12,
@@ -523,6 +604,8 @@ def run_minfer(args):
                          "peak_source": f"bf16_tflops_sustained ({peak_src})",
                          "traffic": traffic,
                          "flops_per_launch": useful},
+            "tensor_pipe": recorded_tensor_pipe(w.name),
+            "at_1m": at_1m,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "dense_prefill": dense,

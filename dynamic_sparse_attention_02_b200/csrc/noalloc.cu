@@ -32,7 +32,9 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // Device address of g_vs_scratch on the current device.  The first call on a
 // device looks it up (cudaGetSymbolAddress, with that device current) and
 // caches it; that first call should therefore happen before any stream
-// capture on that device.
+// capture on that device.  A device reset (cudaDeviceReset) unloads the
+// library's module on that device, so the cached address is no longer the
+// array's: after a reset this entry point must not be used in that process.
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -75,7 +77,9 @@ extern "C" int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, in
     // Nothing in the scratch has to start at zero: every byte the index
     // kernels read is written earlier in the same call, so whatever the last
     // call left there is harmless.
-    return mi_vs_index(q, k, Hq, Hkv, N, d, scale, last_q, vertical_size, slash_size, heads,
-                       n_heads, v_idx, s_idx, v_score, s_score, scratch, kStaticScratchBytes,
-                       stream);
+    rc = mi_vs_index(q, k, Hq, Hkv, N, d, scale, last_q, vertical_size, slash_size, heads,
+                     n_heads, v_idx, s_idx, v_score, s_score, scratch, kStaticScratchBytes, stream);
+    // The capacity check above and mi_vs_index size the scratch the same way;
+    // should they ever disagree, a call that does not fit still reads as one.
+    return rc == MI_ERR_WORKSPACE ? MI_ERR_UNSUPPORTED : rc;
 }

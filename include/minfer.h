@@ -268,6 +268,8 @@ int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v,
  *    it; serialise them, e.g. on one stream.
  *  - The first call on each device looks up the array's device address and
  *    caches it; make that first call before any stream capture on the device.
+ *    A device reset (cudaDeviceReset) invalidates the cached address: do not
+ *    call this entry point again in a process that reset the device.
  * All other arguments, outputs and errors as for mi_vs_index.
  */
 int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int N, int d,

@@ -57,3 +57,19 @@ def test_clamped_and_masked_inputs_are_tiny_and_nonnegative():
     assert np.all(y >= 0) and np.all(y < 2.0 ** -125)
     # flush-to-zero arithmetic reads anything below 2^-126 as zero
     assert np.all(y[:4] < np.finfo(np.float32).tiny)
+
+
+def test_constants_reproduced_by_the_fitting_script():
+    """csrc/fit_exp2.py (Remez exchange, relative error) prints the header's
+    coefficients exactly."""
+    import importlib.util
+    path = os.path.join(os.path.dirname(HDR), "fit_exp2.py")
+    spec = importlib.util.spec_from_file_location("fit_exp2", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    c32, e, e32 = mod.fp32_coefficients(3)
+    k = constants()
+    for j in range(4):
+        assert float(c32[j]) == k[f"kExp2C{j}"], j
+        assert mod.c_hex(c32[j]) in open(HDR).read()
+    assert e < 7.6e-5 and e32 < 7.6e-5

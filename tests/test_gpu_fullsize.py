@@ -4,9 +4,10 @@ against the CPU oracle on seeded heads and rows it can compute one by one.
 
 For each sampled head: the GPU index sets must equal the oracle's except
 within the tie window of the k-th score; the GPU attention fed the oracle's
-own indices must meet max-abs <= 1e-2, mean-abs <= 1e-3 on the sampled rows; and
-where the GPU's index equals the oracle's exactly, the layer's own output at
-those rows must too.
+own indices must meet max-abs <= 1e-2, mean-abs <= 1e-3 on the sampled rows;
+and the layer's own output at those rows must meet the same bound against the
+oracle's attention over the index the layer used: the oracle's own where the
+GPU index equals it, else the GPU's (already checked to differ only at ties).
 """
 import numpy as np
 import pytest
@@ -45,15 +46,17 @@ def check_head(w, x, out_layer, lse_layer, h, rows):
     qs, ks_, vs_ = head_slices(q, k, v, h)
     pt = int(x["pattern"][h])
     same_index = True
+    layer_ref = None  # oracle rows over the GPU's own index, where it differs at ties
     if pt == synth.PATTERN_VS:
         a, b, vert, sl = oracle.vs_index(qs, ks_, 0, w.last_q, w.vertical_size, w.slash_size)
         gv, gs = B.mi_vs_index(q, k, w.last_q, w.vertical_size, w.slash_size, heads=[h])
         torch.cuda.synchronize()
-        same_index &= check_index_set(gv[0].cpu().numpy(), vert, w.vertical_size,
-                                      what=f"vertical h{h}") == 0
-        same_index &= check_index_set(gs[0].cpu().numpy(), sl, w.slash_size,
-                                      what=f"slash h{h}") == 0
+        gva, gsa = gv[0].cpu().numpy(), gs[0].cpu().numpy()
+        same_index &= check_index_set(gva, vert, w.vertical_size, what=f"vertical h{h}") == 0
+        same_index &= check_index_set(gsa, sl, w.slash_size, what=f"slash h{h}") == 0
         ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, a, b, rows=rows)
+        if not same_index:
+            layer_ref = oracle.attn_vs(qs, ks_, vs_, 0, gva[gva >= 0], gsa[gsa >= 0], rows=rows)
         vi = torch.full((1, w.vertical_size), -1, dtype=torch.int32)
         si = torch.full((1, w.slash_size), -1, dtype=torch.int32)
         vi[0, :a.size] = torch.from_numpy(a.astype(np.int32))
@@ -71,6 +74,8 @@ def check_head(w, x, out_layer, lse_layer, h, rows):
                                           window_scale=np.abs(row).max(),
                                           what=f"h{h} bq{bq}") == 0
         ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi, bc, rows=rows)
+        if not same_index:
+            layer_ref = oracle.attn_bs(qs, ks_, vs_, 0, gb, gbc[0].cpu().numpy(), rows=rows)
         out, lse = B.mi_block_sparse_attn(q, k, v, torch.from_numpy(bi[None]).cuda(),
                                           torch.from_numpy(bc[None]).cuda(), heads=[h])
     else:
@@ -81,6 +86,12 @@ def check_head(w, x, out_layer, lse_layer, h, rows):
     check_attn(out[h, ridx], lse[h, ridx], ro, rl, what=f"oracle indices, head {h}")
     if same_index:
         check_attn(out_layer[h, ridx], lse_layer[h, ridx], ro, rl, what=f"layer, head {h}")
+    else:
+        print(f"head {h}: GPU index differs from the oracle's at ties; layer output checked "
+              f"against the oracle over the GPU's index")
+        check_attn(out_layer[h, ridx], lse_layer[h, ridx], layer_ref[0], layer_ref[1],
+                   what=f"layer (GPU index), head {h}")
+    return same_index
 
 
 @pytest.mark.parametrize("name,n_heads,n_rows", [
@@ -99,7 +110,7 @@ def test_full_size_layer_matches_oracle(name, n_heads, n_rows):
         pat = x["pattern"]
         extra = [int(np.nonzero(pat == p_)[0][0]) for p_ in (0, 1, 2)]
         heads = sorted(set(heads) | set(extra))
-    for h in heads:
-        check_head(w, x, out, lse, h, rows)
+    ties = [h for h in heads if not check_head(w, x, out, lse, h, rows)]
+    print(f"{name}: {len(heads)} heads checked, {len(ties)} with index ties {ties}")
     del x, out, lse
     torch.cuda.empty_cache()
