@@ -33,7 +33,7 @@ EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_by
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
            "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
            "mi_vs_index_static", "mi_dense_attn", "mi_prefill_workspace_bytes_heads",
-           "mi_prefill_layer_heads"]
+           "mi_prefill_layer_heads", "mi_debug_set_wait_budget"]
 
 
 class MinferError(RuntimeError):
@@ -86,6 +86,7 @@ def _lib_handle():
         lib.mi_prefill_workspace_bytes_heads.restype = SZ
         lib.mi_prefill_layer_heads.argtypes = [P, P, P, I, I, I, I, F, P, P, P, P, P, P, SZ, P,
                                                P]
+        lib.mi_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
         for name in EXPORTS[5:]:
             if name != "mi_prefill_workspace_bytes_heads":
                 getattr(lib, name).restype = I
@@ -184,6 +185,12 @@ def mi_debug_wait_failure():
     _check("mi_debug_wait_failure", _lib_handle().mi_debug_wait_failure(rec))
     keys = ["seq", "site", "block", "thread", "group", "parity", "r6", "r7"]
     return dict(zip(keys, list(rec)))
+
+
+def mi_debug_set_wait_budget(cycles: int) -> None:
+    """Clock budget of the kernels' abortable waits for later launches
+    (<= 0: the default).  Failure-path tests only."""
+    _check("mi_debug_set_wait_budget", _lib_handle().mi_debug_set_wait_budget(int(cycles)))
 
 
 def mi_status_str(status: int) -> str:

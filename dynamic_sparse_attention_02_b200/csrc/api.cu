@@ -3,16 +3,25 @@
 // the per-head pattern dispatcher of mi_prefill_layer (aifetchly guide,
 // "Phase 2: The Online Dynamic Kernel Router": each head goes to the kernel
 // of its offline-assigned pattern, with no host-device synchronisation).
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 using namespace minfer;
 
 namespace {
 thread_local int g_last_cuda_error = 0;
+std::atomic<long long> g_wait_budget{0};  // 0: the default bound
 }  // namespace
+
+long long minfer::wait_budget_cycles() {
+    const long long b = g_wait_budget.load();
+    return b > 0 ? b : kWaitBudgetCycles;
+}
+void minfer::set_wait_budget_cycles(long long cycles) { g_wait_budget.store(cycles > 0 ? cycles : 0); }
 
 // MI_OK, or MI_ERR_CUDA with the error kept for mi_last_cuda_error().
 int minfer::cuda_status(cudaError_t e) {
@@ -470,6 +479,11 @@ int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v,
                            void* const* stage_events) {
     return prefill_layer(q, k, v, Hq, Hkv, N, d, scale, pattern, params, true, out, lse,
                          err_count, ws, ws_bytes, stream, stage_events);
+}
+
+int mi_debug_set_wait_budget(long long cycles) {
+    set_wait_budget_cycles(cycles);
+    return MI_OK;
 }
 
 int mi_debug_wait_failure(int32_t* record8) {

@@ -112,6 +112,7 @@ __device__ void record_wait_failure(unsigned int seq, int site, int group, int p
 
 struct AttnParams {
     unsigned int seq;  // launch sequence number (never 0)
+    long long wait_budget;  // cycles an abortable wait may take before it gives up
     const bf16* k;
     const bf16* v;
     bf16* out;
@@ -264,7 +265,7 @@ struct Producer {
     // lane 0 waits, the warp follows its verdict
     __device__ bool wait(uint64_t* bar, int parity, int count) {
         bool w = true;
-        if (lane == 0) w = mbar_wait(bar, parity, abort);
+        if (lane == 0) w = mbar_wait(bar, parity, abort, p.wait_budget);
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) {
             if (lane == 0) {
@@ -603,7 +604,7 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
 // So the tensor core computes S(n+1) while the softmax works on S(n).
 template <int D>
 __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int32_t* err,
-                        unsigned int seq, uint32_t tmem, int x) {
+                        unsigned int seq, long long budget, uint32_t tmem, int x) {
     using L = Layout<D>;
     const int lane = threadIdx.x & 31;
     const uint32_t idS = idesc_bf16_f32(128, kChunkKeys, false);
@@ -622,7 +623,7 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
     bool ok = true;
     {
         bool w = true;
-        if (lane == 0) w = mbar_wait(bars.q_full, 0, abort);
+        if (lane == 0) w = mbar_wait(bars.q_full, 0, abort, budget);
         ok = __shfl_sync(0xffffffffu, w, 0);
         if (!ok && lane == 0 && !*abort) record_wait_failure(seq, kSiteMmaQ, 0, x);
     }
@@ -657,7 +658,7 @@ __device__ void run_mma(uint8_t* sm, const Bars& bars, volatile int* abort, int3
         const bool can_s = kv_ready && cnt - (hp ? 1 : 0) <= 1;
         if (!(hp || can_s)) {
             if ((++idle & 15) != 0) continue;
-            const bool give_up = *abort || clock64() - t_last > kWaitBudgetCycles;
+            const bool give_up = *abort || clock64() - t_last > budget;
             if (__any_sync(0xffffffffu, give_up)) {
                 if (lane == 0 && !*abort)
                     record_wait_failure(seq, want_kv ? kSiteMmaFull : kSiteMmaP, g, cnt | x << 4);
@@ -747,7 +748,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     for (int g = 0;; ++g) {
         const int di = g % kDescRing;
         const int dpar = (g / kDescRing) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.desc_full[di], dpar, abort))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.desc_full[di], dpar, abort, p.wait_budget))) {
             if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxFull, g, dpar);
             ok = false;
             break;
@@ -785,7 +786,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                                       (keep != 0 ? 1u : 0u) | (keep != ~0ull ? 2u : 0u));
             const int b = n & 1;
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(&bars.s_full[2 * x + b], (n >> 1) & 1, abort))) {
+                            mbar_wait(&bars.s_full[2 * x + b], (n >> 1) & 1, abort, p.wait_budget))) {
                 if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxS, g, (n >> 1) & 1);
                 ok = false;
                 break;
@@ -833,7 +834,8 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
                     if (n > 0) {
                         const int pb = (n - 1) & 1;
                         if (!__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + pb],
-                                                               ((n - 1) >> 1) & 1, abort))) {
+                                                               ((n - 1) >> 1) & 1, abort,
+                                                               p.wait_budget))) {
                             if (!*abort) record_wait_failure(p.seq, kSiteSoftmaxO, g, 0);
                             ok = false;
                             break;
@@ -886,7 +888,7 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
     bool have = n > 0 && ok;
     if (have) {
         have = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done[2 * x + ((n - 1) & 1)],
-                                                 ((n - 1) >> 1) & 1, abort));
+                                                 ((n - 1) >> 1) & 1, abort, p.wait_budget));
         if (!have && !*abort) record_wait_failure(p.seq, kSiteSoftmaxO, -1, 0);
     }
     if (!ok || (n > 0 && !have)) set_abort(abort, p.err, p.seq);
@@ -1012,7 +1014,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == kProducerWarp) {
             run_producer<D>(p, &tmQ, &tmK, &tmV, sm, bars, abort, patmap, pos, T);
         } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-            run_mma<D>(sm, bars, abort, p.err, p.seq, tmem, warp - kMmaWarp);
+            run_mma<D>(sm, bars, abort, p.err, p.seq, p.wait_budget, tmem, warp - kMmaWarp);
             tc_fence_before();
         }
     }
@@ -1115,6 +1117,7 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
     memset(&p, 0, sizeof(p));
     if (seq == 0) seq = ++next_seq;
     p.seq = seq;
+    p.wait_budget = wait_budget_cycles();
     p.k = a.k;
     p.v = a.v;
     p.out = a.out;

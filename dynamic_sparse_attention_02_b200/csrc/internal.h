@@ -147,4 +147,10 @@ cudaError_t read_wait_failure(int* out8);
 // MI_OK, or MI_ERR_CUDA with the error kept for mi_last_cuda_error().
 int cuda_status(cudaError_t e);
 
+// Clock budget of the abortable in-pipeline waits of the kernels launched from
+// now on (mi_debug_set_wait_budget; default kWaitBudgetCycles of ptx.cuh);
+// teardown waits always keep the full bound.
+long long wait_budget_cycles();
+void set_wait_budget_cycles(long long cycles);
+
 }  // namespace minfer

@@ -97,6 +97,7 @@ struct TcParams {
     int Hq, Hkv, N, L, nchunks, chunk;
     double scale;
     unsigned int seq;
+    long long wait_budget;  // cycles an abortable wait may take before it gives up
     double* m_part;  // pass 1 out: [n_heads][L][nchunks]
     double* l_part;
     const double* mrow;  // pass 2 in: [n_heads][L]
@@ -201,7 +202,7 @@ __device__ void tc_producer(const TcParams& p, const CUtensorMap* tmQ, const CUt
         const int st = t % kTcStages;
         if (t >= kTcStages) {
             const uint32_t par = ((t / kTcStages) - 1) & 1;
-            if (!mbar_wait(&bars.k_empty[st], par, abort)) {
+            if (!mbar_wait(&bars.k_empty[st], par, abort, p.wait_budget)) {
                 if (!*abort) record_vs_wait_failure(p.seq, kSiteTcProducer, t, (int)par);
                 vs_set_abort(abort, p.seq);
                 break;
@@ -233,7 +234,7 @@ __device__ void tc_mma(const TcParams& p, uint8_t* sm, const TcBars& bars, volat
     {
         bool w = true;
         if (lane == 0) {
-            w = mbar_wait(bars.q_full, 0, abort);
+            w = mbar_wait(bars.q_full, 0, abort, p.wait_budget);
             if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaQ, 0, 0);
         }
         ok = __shfl_sync(0xffffffffu, w, 0);
@@ -243,11 +244,11 @@ __device__ void tc_mma(const TcParams& p, uint8_t* sm, const TcBars& bars, volat
         bool w = true;
         if (lane == 0) {
             const uint32_t kpar = (t / kTcStages) & 1;
-            w = mbar_wait(&bars.k_full[st], kpar, abort);
+            w = mbar_wait(&bars.k_full[st], kpar, abort, p.wait_budget);
             if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaK, t, (int)kpar);
             if (w && t >= 2) {
                 const uint32_t apar = ((t >> 1) - 1) & 1;
-                w = mbar_wait(&bars.acc_empty[b], apar, abort);
+                w = mbar_wait(&bars.acc_empty[b], apar, abort, p.wait_budget);
                 if (!w && !*abort) record_vs_wait_failure(p.seq, kSiteTcMmaAcc, t, (int)apar);
             }
         }
@@ -281,7 +282,7 @@ __device__ __forceinline__ bool epi_wait(const TcParams& p, const TcBars& bars,
     bool w = true;
     if (lane == 0) {
         const uint32_t par = (t >> 1) & 1;
-        w = mbar_wait(&bars.acc_full[t & 1], par, abort);
+        w = mbar_wait(&bars.acc_full[t & 1], par, abort, p.wait_budget);
         if (!w) {
             if (!*abort) record_vs_wait_failure(p.seq, kSiteTcEpilogue, t, (int)par);
             vs_set_abort(abort, p.seq);
@@ -680,6 +681,7 @@ cudaError_t launch_vs_scores_tc(int pass, const bf16* q, const bf16* k, int Hq, 
     memset(&p, 0, sizeof(p));
     if (seq == 0) seq = ++next_seq;
     p.seq = seq;
+    p.wait_budget = wait_budget_cycles();
     p.heads = heads;
     // items of each KV head in list order (each head's row groups together),
     // paired into tiles; an odd one out runs alone

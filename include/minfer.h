@@ -293,6 +293,19 @@ int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int 
  */
 int mi_debug_wait_failure(int32_t* record8);
 
+/*
+ * Diagnostics: the clock budget (in SM cycles) of every abortable wait inside
+ * the kernels launched after this call; cycles <= 0 restores the default of
+ * about half a second.  Waits that guard the release of tensor memory or the
+ * landing of copies in flight keep the full budget whatever is set here, so
+ * a launch whose waits give up still ends cleanly: it sets bit 30 of its
+ * err_count, records the site for mi_debug_wait_failure, writes zero rows,
+ * and leaves the device usable.  For tests of that failure path only; a
+ * small budget makes correct launches give up.  Process-wide, not thread-safe
+ * against concurrent launches.
+ */
+int mi_debug_set_wait_budget(long long cycles);
+
 #ifdef __cplusplus
 }
 #endif
