@@ -48,7 +48,7 @@ def log(msg):
 
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SOURCES = ["attn.cu", "ptx.cuh", "internal.h"]
+ATTN_SOURCES = ["attn.cu", "attn_kt.cu", "softmax_math.cuh", "exp2_poly.h", "ptx.cuh", "internal.h"]
 
 
 def parse_args(argv=None):

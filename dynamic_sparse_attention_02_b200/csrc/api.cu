@@ -279,7 +279,8 @@ int mi_block_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, i
     a.blk_idx = blk_idx;
     a.blk_cnt = blk_cnt;
     a.topk = topk;
-    return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_status(kt_attn_supported(a) ? launch_kt_attn(a, st) : launch_sparse_attn(a, st));
 }
 
 int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
@@ -446,6 +447,18 @@ int prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, 
     a.sink_h = lp.sink_h;
     a.window_h = lp.win_h;
     a.n_asw = lp.n_a;
+    // Block-Sparse heads run on the key-major engine where it applies, the
+    // rest (and all heads otherwise) in one launch of the row-major engine
+    if (lp.bs.n && kt_attn_supported(a)) {
+        AttnLaunch abs = a;
+        abs.heads.n = 0;
+        a.heads.n = 0;
+        for (int i = 0; i < lp.all.n; ++i) {
+            HeadList& dst = head_pattern(lp.all.e[i]) == MI_PATTERN_BS ? abs.heads : a.heads;
+            dst.e[dst.n++] = lp.all.e[i];
+        }
+        if ((rc = cuda_status(launch_kt_attn(abs, st)))) return rc;
+    }
     if ((rc = cuda_status(launch_sparse_attn(a, st)))) return rc;
     return rec(MI_STAGE_ATTN_DONE);
 }
@@ -488,14 +501,17 @@ int mi_debug_set_wait_budget(long long cycles) {
 
 int mi_debug_wait_failure(int32_t* record8) {
     if (!record8) return MI_ERR_INVALID_ARG;
-    // attention's record first, else the tensor-core VS score passes' (sites >= 11);
-    // reading clears both
-    int rec[8], rec_vs[8];
+    // the row-major attention record first, then the key-major attention one
+    // (sites 21..27), else the tensor-core VS score passes' (sites 11..15);
+    // reading clears all three
+    int rec[8], rec_kt[8], rec_vs[8];
     int rc = cuda_status(read_wait_failure(rec));
+    if (rc) return rc;
+    rc = cuda_status(read_kt_wait_failure(rec_kt));
     if (rc) return rc;
     rc = cuda_status(read_vs_wait_failure(rec_vs));
     if (rc) return rc;
-    const int* use = rec[1] != 0 ? rec : rec_vs;
+    const int* use = rec[1] != 0 ? rec : (rec_kt[1] != 0 ? rec_kt : rec_vs);
     for (int i = 0; i < 8; ++i) record8[i] = use[i];
     return MI_OK;
 }

@@ -139,6 +139,11 @@ struct AttnLaunch {
     int32_t* err_count;
 };
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t st);
+// Block-Sparse heads on key-major tiles (attn_kt.cu): d = 128 and N up to
+// about 8M (its per-item block bitmap lives in shared memory).
+bool kt_attn_supported(const AttnLaunch& a);
+cudaError_t launch_kt_attn(const AttnLaunch& a, cudaStream_t st);
+cudaError_t read_kt_wait_failure(int* out8);
 // 2-D TMA map over a [rows][d] bf16 matrix: boxes of 64 columns x box_rows
 // rows, 128-byte swizzle, zero fill past the last row.
 bool make_tma_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows);

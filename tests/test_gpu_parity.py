@@ -125,7 +125,9 @@ def test_ashape_attn_matches_oracle(Hq, Hkv, N, d, sink, window):
 
 
 @pytest.mark.parametrize("Hq,Hkv,N,d,topk", [
-    (4, 1, 1024, 128, 4), (2, 2, 576, 64, 3), (2, 1, 2048, 128, 100)])
+    (4, 1, 1024, 128, 4), (2, 2, 576, 64, 3), (2, 1, 2048, 128, 100),
+    (6, 2, 4096, 128, 9),    # more items than one CTA per SM takes at once, odd topk
+    (1, 1, 64, 128, 1)])     # a single query block
 def test_block_sparse_attn_matches_oracle(Hq, Hkv, N, d, topk):
     q, k, v = rand_bf16(Hq, Hkv, N, d, 12)
     nB = N // 64
@@ -141,6 +143,79 @@ def test_block_sparse_attn_matches_oracle(Hq, Hkv, N, d, topk):
     torch.cuda.synchronize()
     for h in range(Hq):
         check_attn(out[h], lse[h], *refs[h], what=f"bs h{h}")
+
+
+def test_block_sparse_attn_unusual_lists_and_empty_rows():
+    """Block lists as a caller may pass them: unsorted, with duplicates, -1
+    padding in the middle, entries past the query block or outside [0, N/64)
+    (skipped and counted), counts above topk (clamped to topk) and rows with no
+    block at all (out 0, lse -inf).  Odd counts leave half of a key-major tile
+    unused; query blocks whose own block is chosen need the causal mask."""
+    Hq, Hkv, N, d, topk = 4, 2, 1536, 128, 7
+    q, k, v = rand_bf16(Hq, Hkv, N, d, 61)
+    nB = N // 64
+    rng = np.random.default_rng(3)
+    bi = np.full((Hq, nB, topk), -1, np.int32)
+    bc = np.zeros((Hq, nB), np.int32)
+    for h in range(Hq):
+        for bq in range(nB):
+            c = int(rng.integers(0, topk + 3))  # above topk: clamped
+            row = rng.integers(0, bq + 1, size=topk).astype(np.int32)
+            for t in range(topk):
+                r = rng.random()
+                if r < 0.1:
+                    row[t] = -1                    # padding, not counted
+                elif r < 0.15:
+                    row[t] = bq + 1 + int(rng.integers(0, 3))  # past the query block
+                elif r < 0.18:
+                    row[t] = -5                    # negative, not padding
+            bi[h, bq], bc[h, bq] = row, c
+    bc[0, 3] = 0                     # an empty query block
+    bi[1, 5, :] = -1                 # only padding: empty too
+    bc[1, 5] = topk
+    n_bad = 0
+    for h in range(Hq):
+        for bq in range(nB):
+            for t in range(min(int(bc[h, bq]), topk)):
+                e = int(bi[h, bq, t])
+                n_bad += e != -1 and (e < 0 or e > bq)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = B.mi_block_sparse_attn(q, k, v, torch.from_numpy(bi).cuda(),
+                                      torch.from_numpy(bc).cuda(), err_count=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == n_bad
+    for h in range(Hq):
+        qs, ks_, vs_ = head_slices(q, k, v, h)
+        ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi[h], bc[h])
+        check_attn(out[h], lse[h], ro, rl, what=f"bs lists h{h}")
+    assert (out[0, 192:256] == 0).all() and torch.isneginf(lse[0, 192:256]).all()
+
+
+def test_block_sparse_attn_rescales_mid_item():
+    """A query block whose later key blocks score far above its first ones:
+    the per-query reference max must move up mid-item (the lazy rescale of
+    O and of the running sums), and a block scoring far below must not."""
+    Hq, Hkv, N, d = 2, 1, 1024, 128
+    q, k, v = rand_bf16(Hq, Hkv, N, d, 62)
+    q, k = q.clone(), k.clone()
+    qd = q[:, 640:704].float().mean(dim=(0, 1))
+    k[0, 320:384] = (100.0 * qd / qd.norm()).to(torch.bfloat16)   # block 5: large scores
+    k[0, 128:192] = (-100.0 * qd / qd.norm()).to(torch.bfloat16)  # block 2: tiny weights
+    nB, topk = N // 64, 6
+    bi = np.full((Hq, nB, topk), -1, np.int32)
+    bc = np.zeros((Hq, nB), np.int32)
+    for h in range(Hq):
+        for bq in range(nB):
+            lst = sorted({0, bq, bq // 2, 2 if bq >= 2 else 0, 5 if bq >= 5 else 0})
+            bi[h, bq, :len(lst)] = lst
+            bc[h, bq] = len(lst)
+    out, lse = B.mi_block_sparse_attn(q, k, v, torch.from_numpy(bi).cuda(),
+                                      torch.from_numpy(bc).cuda())
+    torch.cuda.synchronize()
+    for h in range(Hq):
+        qs, ks_, vs_ = head_slices(q, k, v, h)
+        ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi[h], bc[h])
+        check_attn(out[h], lse[h], ro, rl, what=f"bs rescale h{h}")
 
 
 @pytest.mark.parametrize("Hq,Hkv,N,d,L,kv,ks", [
