@@ -55,6 +55,9 @@ def _load():
                                                 I64, P, P]
             lib.oracle_attn_bs_rows.argtypes = [P, P, P, I, I, I, I, D, I, P, P, I, I, P, I64, P,
                                                 P]
+            lib.oracle_attn_vs_range_rows.argtypes = [P, P, P, I, I, I, I, D, I, P, I64, P, I64,
+                                                      I, P, I64, P, P]
+            lib.oracle_vs_mask.argtypes = [I, P, I64, P, I64, I, I, P]
             lib.oracle_num_threads.restype = I
             _lib = lib
     return _lib
@@ -172,6 +175,29 @@ def attn_vs(q, k, v, h, v_idx, s_idx, rows=None, block=64, scale=None):
                                        _ptr(vi), vi.size, _ptr(si), si.size, block, _ptr(rows),
                                        rows.size, _ptr(out), _ptr(lse)), "vs")
     return out, lse
+
+
+def attn_vs_range(q, k, v, h, v_idx, s_idx, rows=None, block=64, scale=None):
+    """Vertical-Slash attention rows with range-based slash tiles: diagonal o
+    covers keys [64 bq - o, 64 bq + 63 - o] for query block bq."""
+    q, k, v, Hq, Hkv, N, d, rows, out, lse = _attn_common(q, k, v, rows)
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    vi, si = _i32(v_idx), _i32(s_idx)
+    _check(_load().oracle_attn_vs_range_rows(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale, h,
+                                             _ptr(vi), vi.size, _ptr(si), si.size, block,
+                                             _ptr(rows), rows.size, _ptr(out), _ptr(lse)),
+           "vs_range")
+    return out, lse
+
+
+def vs_mask(N, v_idx, s_idx, range_tiles=False, block=64):
+    """The causal Vertical-Slash mask, bool [N, N]: whole 64x64 slash tiles, or
+    range-based ones (range_tiles=True)."""
+    vi, si = _i32(v_idx), _i32(s_idx)
+    m = np.zeros((N, N), np.uint8)
+    _check(_load().oracle_vs_mask(N, _ptr(vi), vi.size, _ptr(si), si.size, block,
+                                  1 if range_tiles else 0, _ptr(m)), "vs_mask")
+    return m.astype(bool)
 
 
 def attn_bs(q, k, v, h, blk_idx, blk_cnt, rows=None, block=64, scale=None):

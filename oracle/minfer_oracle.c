@@ -421,6 +421,103 @@ int oracle_attn_vs_rows(const float* q, const float* k, const float* v, int Hq, 
     return rc;
 }
 
+/* Vertical-Slash with range-based slash tiles (aifetchly guide, "2. The   */
+/* Vertical-Slash Pattern": the diagonals cost O(N (k_v + k_s)) rather than */
+/* whole tiles).  For the 64-row query block bq of row i, diagonal o covers  */
+/* the unaligned 64-key range [64 bq - o, 64 bq + 63 - o]; key j is kept     */
+/* for row i iff j is a selected column or j lies in the range of some       */
+/* selected diagonal.                                                        */
+typedef struct {
+    const uint8_t* in_v;   /* [N] selected columns */
+    const int64_t* s_cnt;  /* [N + 1]: s_cnt[x] = number of selected diagonals o < x */
+    int64_t N;
+    int block;
+} vsr_ctx;
+
+static int allow_vs_range(const void* ctx, int64_t i, int64_t j) {
+    const vsr_ctx* c = (const vsr_ctx*)ctx;
+    if (c->in_v[j]) return 1;
+    const int64_t base = (i / c->block) * c->block; /* 64 bq */
+    /* j in [base - o, base + block - 1 - o]  <=>  o in [base - j, base + block - 1 - j] */
+    int64_t lo = base - j, hi = base + c->block - 1 - j;
+    if (lo < 0) lo = 0;
+    if (hi > c->N - 1) hi = c->N - 1;
+    if (lo > hi) return 0;
+    return c->s_cnt[hi + 1] - c->s_cnt[lo] > 0;
+}
+
+/* in_v [N] and s_cnt [N + 1] from the index lists (entries outside [0, N) ignored). */
+static int vs_range_tables(int N, const int32_t* v_idx, int64_t kv, const int32_t* s_idx,
+                           int64_t ks, uint8_t** in_v, int64_t** s_cnt) {
+    *in_v = (uint8_t*)calloc((size_t)N, 1);
+    *s_cnt = (int64_t*)calloc((size_t)N + 1, sizeof(int64_t));
+    uint8_t* in_s = (uint8_t*)calloc((size_t)N, 1);
+    if (!*in_v || !*s_cnt || !in_s) {
+        free(*in_v);
+        free(*s_cnt);
+        free(in_s);
+        return ORACLE_ENOMEM;
+    }
+    for (int64_t t = 0; t < kv; ++t)
+        if (v_idx[t] >= 0 && v_idx[t] < N) (*in_v)[v_idx[t]] = 1;
+    for (int64_t t = 0; t < ks; ++t)
+        if (s_idx[t] >= 0 && s_idx[t] < N) in_s[s_idx[t]] = 1;
+    for (int64_t x = 0; x < N; ++x) (*s_cnt)[x + 1] = (*s_cnt)[x] + in_s[x];
+    free(in_s);
+    return ORACLE_OK;
+}
+
+int oracle_attn_vs_range_rows(const float* q, const float* k, const float* v, int Hq, int Hkv,
+                              int N, int d, double scale, int h, const int32_t* v_idx,
+                              int64_t kv, const int32_t* s_idx, int64_t ks, int block,
+                              const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    if (check_attn_args(q, k, v, Hq, Hkv, N, d, h, rows, n_rows, out, lse) || kv < 0 ||
+        ks < 0 || (!v_idx && kv > 0) || (!s_idx && ks > 0) || block <= 0 || N % block)
+        return ORACLE_EINVAL;
+    uint8_t* in_v;
+    int64_t* s_cnt;
+    int rc = vs_range_tables(N, v_idx, kv, s_idx, ks, &in_v, &s_cnt);
+    if (rc) return rc;
+    vsr_ctx c = {in_v, s_cnt, N, block};
+    rc = attn_rows(q, k, v, Hq, Hkv, N, d, scale, h, allow_vs_range, &c, rows, n_rows, out, lse);
+    free(in_v);
+    free(s_cnt);
+    return rc;
+}
+
+/* The causal Vertical-Slash mask itself, mask[i][j] for 0 <= i, j < N (1 =    */
+/* kept): whole 64x64 tiles (range = 0) or range-based slash tiles            */
+/* (range = 1).  For the pins only (N x N bytes).                              */
+int oracle_vs_mask(int N, const int32_t* v_idx, int64_t kv, const int32_t* s_idx, int64_t ks,
+                   int block, int range, uint8_t* mask) {
+    if (N <= 0 || block <= 0 || N % block || kv < 0 || ks < 0 || (!v_idx && kv > 0) ||
+        (!s_idx && ks > 0) || !mask)
+        return ORACLE_EINVAL;
+    uint8_t* in_v;
+    int64_t* s_cnt;
+    int rc = vs_range_tables(N, v_idx, kv, s_idx, ks, &in_v, &s_cnt);
+    if (rc) return rc;
+    uint8_t* D = (uint8_t*)calloc((size_t)(N / block), 1);
+    if (!D) {
+        free(in_v);
+        free(s_cnt);
+        return ORACLE_ENOMEM;
+    }
+    rc = oracle_slash_deltas(s_idx, ks, N, block, D);
+    if (rc == ORACLE_OK) {
+        vs_ctx ca = {in_v, D, block};
+        vsr_ctx cr = {in_v, s_cnt, N, block};
+        for (int64_t i = 0; i < N; ++i)
+            for (int64_t j = 0; j < N; ++j)
+                mask[(size_t)i * N + j] =
+                    (uint8_t)(j <= i && (range ? allow_vs_range(&cr, i, j) : allow_vs(&ca, i, j)));
+    }
+    free(in_v);
+    free(s_cnt);
+    free(D);
+    return rc;
+}
+
 /* Block-Sparse: key j kept for row i iff bk(j) is listed for bq(i). */
 typedef struct {
     const uint8_t* sel; /* [nB][nB], sel[bq*nB + bk] */

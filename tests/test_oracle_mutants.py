@@ -58,6 +58,14 @@ MUTANTS = [
      "lse[r] = m + log(l);", "lse[r] = log(l);"),
     ("vs_attn_delta_from_key_block_only",
      "return c->D[i / c->block - j / c->block] != 0;", "return c->D[j / c->block] != 0;"),
+    ("vs_range_upper_bound_off_by_one",
+     "int64_t lo = base - j, hi = base + c->block - 1 - j;",
+     "int64_t lo = base - j, hi = base + c->block - j;"),
+    ("vs_range_from_the_row_not_its_block",
+     "const int64_t base = (i / c->block) * c->block; /* 64 bq */",
+     "const int64_t base = i; /* 64 bq */"),
+    ("vs_range_prefix_count_shifted",
+     "return c->s_cnt[hi + 1] - c->s_cnt[lo] > 0;", "return c->s_cnt[hi] - c->s_cnt[lo] > 0;"),
     ("bs_attn_block_table_transposed",
      "return c->sel[(size_t)(i / c->block) * c->nB + (size_t)(j / c->block)] != 0;",
      "return c->sel[(size_t)(j / c->block) * c->nB + (size_t)(i / c->block)] != 0;"),

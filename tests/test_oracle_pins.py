@@ -412,3 +412,83 @@ def test_attention_hand_worked(c):
     empty = lse_of == 0
     assert np.all(np.isneginf(lse[empty]))
     np.testing.assert_allclose(lse[~empty], np.log(lse_of[~empty]), rtol=1e-14, atol=1e-15)
+
+
+# ------------------------------------------- range-based slash tiles (§ next)
+
+def _brute_range_mask(N, v_idx, s_idx, block=64):
+    """The range predicate built diagonal by diagonal: for every selected o and
+    every query block bq, mark keys [64 bq - o, 64 bq + 63 - o] for the rows of
+    bq; then the selected columns; then the causal limit."""
+    m = np.zeros((N, N), bool)
+    for o in s_idx:
+        if not 0 <= o < N:
+            continue
+        for bq in range(N // block):
+            lo, hi = max(0, block * bq - o), block * bq + block - 1 - o
+            if hi >= lo:
+                m[block * bq:block * bq + block, lo:hi + 1] = True
+    for c in v_idx:
+        if 0 <= c < N:
+            m[:, c] = True
+    return m & np.tril(np.ones((N, N), bool))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_vs_range_mask_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    N = 512
+    s_idx = rng.choice(N, size=12, replace=False).astype(np.int32)
+    v_idx = rng.choice(N, size=5, replace=False).astype(np.int32)
+    got = oracle.vs_mask(N, v_idx, s_idx, range_tiles=True)
+    np.testing.assert_array_equal(got, _brute_range_mask(N, v_idx, s_idx))
+
+
+def test_vs_range_between_exact_diagonals_and_whole_tiles():
+    """Exact diagonals (j = i - o) lie inside the ranges, which lie inside the
+    whole 64x64 tiles the same diagonals touch; equality on neither side."""
+    rng = np.random.default_rng(5)
+    N = 640
+    s_idx = rng.choice(N, size=20, replace=False).astype(np.int32)
+    rng_m = oracle.vs_mask(N, [], s_idx, range_tiles=True)
+    tile_m = oracle.vs_mask(N, [], s_idx, range_tiles=False)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    exact = (j <= i) & np.isin(i - j, s_idx)
+    assert np.all(rng_m[exact]) and np.all(tile_m[rng_m])
+    assert rng_m.sum() > exact.sum() and tile_m.sum() > rng_m.sum()
+
+
+def test_vs_range_hand_cases():
+    """Worked by hand, N = 192 (three query blocks), no columns:
+    o = 0 -> each query block takes its own block (causal);
+    o = 64 -> each query block takes the previous block whole, block 0 none;
+    o = 1 -> query block bq takes keys 64 bq - 1 .. 64 bq + 62."""
+    N = 192
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    bq = i // 64
+    m0 = oracle.vs_mask(N, [], [0], range_tiles=True)
+    np.testing.assert_array_equal(m0, (j // 64 == bq) & (j <= i))
+    m64 = oracle.vs_mask(N, [], [64], range_tiles=True)
+    np.testing.assert_array_equal(m64, j // 64 == bq - 1)
+    m1 = oracle.vs_mask(N, [], [1], range_tiles=True)
+    np.testing.assert_array_equal(m1, (j >= 64 * bq - 1) & (j <= 64 * bq + 62) & (j <= i))
+
+
+def test_vs_range_attention_matches_sdpa_with_the_mask():
+    Hq, Hkv, N, d = 2, 1, 384, 64
+    q, k, v = rand_qkv(Hq, Hkv, N, d, 17)
+    v_idx = np.array([2, 90, 300], np.int32)
+    s_idx = np.array([0, 33, 130, 200], np.int32)
+    mask = _brute_range_mask(N, v_idx, s_idx)
+    out, lse = oracle.attn_vs_range(q, k, v, 1, v_idx, s_idx)
+    np.testing.assert_allclose(out, sdpa_rows(q, k, v, 1, mask=mask), atol=1e-12)
+
+
+def test_vs_range_full_slash_budget_is_dense():
+    """Every diagonal selected: every causal key is covered (P1 for ranges)."""
+    Hq, Hkv, N, d = 1, 1, 256, 64
+    q, k, v = rand_qkv(Hq, Hkv, N, d, 18)
+    out, _ = oracle.attn_vs_range(q, k, v, 0, [], np.arange(N))
+    np.testing.assert_allclose(out, sdpa_rows(q, k, v, 0, causal=True), atol=1e-12)
