@@ -434,9 +434,14 @@ __device__ void kt_run_mma(const KtParams& p, uint8_t* sm, const KtBars& bars,
             !wait(&bars.o_free[pend_o & 1], ((pend_o >> 1) - 1) & 1, kSiteKtMmaP, m))
             return;
         tc_fence_after();
-        const uint32_t vst = v_addr + (m % kKtVStages) * KtLayout::kKVBytes;
-        const uint32_t pst = p_addr + b * KtLayout::kPBytes;
-        const uint32_t tO = tmem + 128 + 64 * (pend_o & 1);
+        // Every operand is broadcast from lane 0 so that the compiler keeps it in
+        // a uniform register: an MMA whose operands it cannot prove warp-uniform
+        // issues several times slower than the tensor pipe runs.
+        const uint32_t vst =
+            __shfl_sync(0xffffffffu, v_addr + (m % kKtVStages) * KtLayout::kKVBytes, 0);
+        const uint32_t pst = __shfl_sync(0xffffffffu, p_addr + b * KtLayout::kPBytes, 0);
+        const uint32_t tO = __shfl_sync(0xffffffffu, tmem + 128 + 64 * (pend_o & 1), 0);
+        const uint32_t acc0 = __shfl_sync(0xffffffffu, (pend_flags & kKtFirst) ? 0u : 1u, 0);
 #pragma unroll
         for (int kk = 0; kk < kKtKeys / 16; ++kk) {
             // A = V^T (d x keys) stored MN-major: d-panels of 64 at kPanelKV apart,
@@ -444,7 +449,7 @@ __device__ void kt_run_mma(const KtParams& p, uint8_t* sm, const KtBars& bars,
             const uint64_t adesc = sw128_desc(vst + kk * 2048, KtLayout::kPanelKV, 1024);
             // B = P^T (64 queries x keys) stored MN-major: one 128-byte row per key
             const uint64_t bdesc = sw128_desc(pst + kk * 2048, KtLayout::kPBytes, 1024);
-            mma_ss_warp(tO, adesc, bdesc, idO, ((pend_flags & kKtFirst) && kk == 0) ? 0u : 1u);
+            mma_ss_warp(tO, adesc, bdesc, idO, kk == 0 ? acc0 : 1u);
         }
         mma_commit_warp(&bars.p_free[b]);
         mma_commit_warp(&bars.v_empty[m % kKtVStages]);
@@ -472,8 +477,9 @@ __device__ void kt_run_mma(const KtParams& p, uint8_t* sm, const KtBars& bars,
         if (!wait(&bars.k_full[n % kKtKStages], (n / kKtKStages) & 1, kSiteKtMmaK, n)) break;
         if (n >= 2 && !wait(&bars.p_full[n & 1], ((n - 2) >> 1) & 1, kSiteKtMmaP, n)) break;
         tc_fence_after();
-        const uint32_t kst = k_addr + (n % kKtKStages) * KtLayout::kKVBytes;
-        const uint32_t tS = tmem + 64 * (n & 1);
+        const uint32_t kst =
+            __shfl_sync(0xffffffffu, k_addr + (n % kKtKStages) * KtLayout::kKVBytes, 0);
+        const uint32_t tS = __shfl_sync(0xffffffffu, tmem + 64 * (n & 1), 0);
 #pragma unroll
         for (int kk = 0; kk < kKtD / 16; ++kk) {
             const int pn = kk >> 2, off = (kk & 3) * 32;
