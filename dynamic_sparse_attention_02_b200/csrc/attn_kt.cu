@@ -399,6 +399,18 @@ __device__ void kt_run_producer(const KtParams& p, const CUtensorMap* tmQ, const
 }
 
 // ------------------------------------------------------------- MMA issuer
+// One converged warp.  An mbarrier probe costs a couple of hundred cycles
+// even on a completed phase, so each round tests every barrier the next
+// actions need in ONE non-blocking test_wait across lanes, then issues what is
+// ready:
+//   lane 0  the next descriptor            lane 4  P^T of the oldest pending O
+//   lane 1  K of the next S                lane 5  V of that chunk
+//   lane 2  its S^T buffer free            lane 6  its O^T buffer free (first
+//   lane 3  the item's Q (first chunk)             chunk of an item two back)
+// S^T of chunk n goes first (it feeds the softmax), then O^T of the oldest
+// chunk whose P^T is ready.  All MMA operands come from lane-0 broadcasts, so
+// they stay in uniform registers (operands the compiler cannot prove uniform
+// make each MMA issue several times slower than the tensor pipe runs).
 __device__ void kt_run_mma(const KtParams& p, uint8_t* sm, const KtBars& bars,
                            volatile int* abort, uint32_t tmem) {
     const int lane = threadIdx.x & 31;
@@ -410,93 +422,115 @@ __device__ void kt_run_mma(const KtParams& p, uint8_t* sm, const KtBars& bars,
     const uint32_t v_addr = __shfl_sync(0xffffffffu, smem_u32(sm + KtLayout::v_off), 0);
     const uint32_t p_addr = __shfl_sync(0xffffffffu, smem_u32(sm + KtLayout::p_off), 0);
     const KtDesc* desc = reinterpret_cast<const KtDesc*>(sm + KtLayout::desc_off);
-    bool ok = true;
 
-    auto wait = [&](uint64_t* bar, int parity, int site, int chunk) -> bool {
-        bool w = true;
-        if (lane == 0) {
-            w = mbar_wait(bar, parity, abort, p.wait_budget);
-            if (!w && !*abort) kt_record_wait_failure(p.seq, site, chunk, parity);
+    // chunks whose S^T has run but not their O^T yet (at most three), 8 bits
+    // each at (chunk % 4) * 8: descriptor flags, O^T buffer parity (bit 5),
+    // O^T buffer last used by an item two back (bit 6)
+    uint32_t pend = 0;
+    int nd = 0;            // next descriptor
+    bool have = false;     // descriptor read, its S^T not issued yet
+    int dflags = 0;
+    int ns = 0, no = 0;    // next S^T / O^T chunk
+    int qi = 0, cur_o = 0; // items with chunks so far; the current one's O^T index
+    bool done = false, ok = true;
+    unsigned idle = 0;
+    long long t_last = clock64();
+    while (ok && !(done && no == ns)) {
+        const uint32_t po = (pend >> ((no & 3) * 8)) & 0xFFu;
+        uint64_t* bar = bars.q_full;  // a completed barrier for lanes with nothing to test
+        uint32_t par = 0;
+        bool live = false;
+        if (lane == 0 && !have && !done) {
+            bar = &bars.desc_full[nd % kKtDescRing]; par = (nd / kKtDescRing) & 1; live = true;
+        } else if (lane == 1 && have) {
+            bar = &bars.k_full[ns % kKtKStages]; par = (ns / kKtKStages) & 1; live = true;
+        } else if (lane == 2 && have && ns >= 2) {
+            bar = &bars.p_full[ns & 1]; par = ((ns - 2) >> 1) & 1; live = true;
+        } else if (lane == 3 && have && (dflags & kKtFirst)) {
+            bar = bars.q_full; par = qi & 1; live = true;
+        } else if (lane == 4 && no < ns) {
+            bar = &bars.p_full[no & 1]; par = (no >> 1) & 1; live = true;
+        } else if (lane == 5 && no < ns) {
+            bar = &bars.v_full[no % kKtVStages]; par = (no / kKtVStages) & 1; live = true;
+        } else if (lane == 6 && no < ns && (po & kKtFirst) && (po & 64)) {
+            // the O^T buffer was last used by the item two back: its epilogue
+            // (completion (item / 2) - 1 of that buffer's o_free) must have read it
+            bar = &bars.o_free[(po >> 5) & 1];
+            par = ((po >> 7) & 1) ^ 1;
+            live = true;
         }
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) ok = false;
-        return w;
-    };
-
-    // O^T += V^T P^T for chunk m (item buffer o; first / last of its item)
-    int pend = -1, pend_flags = 0, pend_o = 0;
-    auto issue_o = [&]() {
-        if (pend < 0 || !ok) return;
-        const int m = pend, b = m & 1;
-        if (!wait(&bars.p_full[b], (m >> 1) & 1, kSiteKtMmaP, m)) return;
-        if (!wait(&bars.v_full[m % kKtVStages], (m / kKtVStages) & 1, kSiteKtMmaK, m)) return;
-        if ((pend_flags & kKtFirst) && pend_o >= 2 &&
-            !wait(&bars.o_free[pend_o & 1], ((pend_o >> 1) - 1) & 1, kSiteKtMmaP, m))
-            return;
-        tc_fence_after();
-        // Every operand is broadcast from lane 0 so that the compiler keeps it in
-        // a uniform register: an MMA whose operands it cannot prove warp-uniform
-        // issues several times slower than the tensor pipe runs.
-        const uint32_t vst =
-            __shfl_sync(0xffffffffu, v_addr + (m % kKtVStages) * KtLayout::kKVBytes, 0);
-        const uint32_t pst = __shfl_sync(0xffffffffu, p_addr + b * KtLayout::kPBytes, 0);
-        const uint32_t tO = __shfl_sync(0xffffffffu, tmem + 128 + 64 * (pend_o & 1), 0);
-        const uint32_t acc0 = __shfl_sync(0xffffffffu, (pend_flags & kKtFirst) ? 0u : 1u, 0);
-#pragma unroll
-        for (int kk = 0; kk < kKtKeys / 16; ++kk) {
-            // A = V^T (d x keys) stored MN-major: d-panels of 64 at kPanelKV apart,
-            // 16 keys = 16 rows of 128 bytes per K-step
-            const uint64_t adesc = sw128_desc(vst + kk * 2048, KtLayout::kPanelKV, 1024);
-            // B = P^T (64 queries x keys) stored MN-major: one 128-byte row per key
-            const uint64_t bdesc = sw128_desc(pst + kk * 2048, KtLayout::kPBytes, 1024);
-            mma_ss_warp(tO, adesc, bdesc, idO, kk == 0 ? acc0 : 1u);
-        }
-        mma_commit_warp(&bars.p_free[b]);
-        mma_commit_warp(&bars.v_empty[m % kKtVStages]);
-        if (pend_flags & kKtLast) mma_commit_warp(&bars.o_full[pend_o & 1]);
-        pend = -1;
-    };
-
-    int nc = 0, qi = 0, cur_o = 0;
-    for (int nd = 0; ok; ++nd) {
-        const int slot = nd % kKtDescRing;
-        if (!wait(&bars.desc_full[slot], (nd / kKtDescRing) & 1, kSiteKtMmaQ, -1 - nd)) break;
-        const int type = __shfl_sync(0xffffffffu, desc[slot].type, 0);
-        const int flags = __shfl_sync(0xffffffffu, desc[slot].flags, 0);
-        if (type != kKtChunk) {
-            mbar_arrive_warp(&bars.desc_empty[slot]);
-            if (type == kKtEnd) break;
+        const bool hit = live ? mbar_test_wait(bar, par) : true;
+        const unsigned bal = __ballot_sync(0xffffffffu, hit);
+        const bool desc_ready = !have && !done && (bal & 1u);
+        const bool s_ready = have && ((bal >> 1) & 7u) == 7u;
+        const bool o_ready = no < ns && ((bal >> 4) & 7u) == 7u;
+        if (!(desc_ready || s_ready || o_ready)) {
+            if ((++idle & 15) != 0) continue;
+            const bool give_up = *abort || clock64() - t_last > p.wait_budget;
+            if (__any_sync(0xffffffffu, give_up)) {
+                if (lane == 0 && !*abort)
+                    kt_record_wait_failure(p.seq, have ? kSiteKtMmaK : kSiteKtMmaP, ns, no);
+                ok = false;
+            }
             continue;
         }
-        const int n = nc++;
-        if (flags & kKtFirst) {
-            issue_o();  // finish the previous item before waiting for this one's Q
-            if (!wait(bars.q_full, qi & 1, kSiteKtMmaQ, n)) break;
-            cur_o = qi++;
+        t_last = clock64();
+        if (desc_ready) {
+            const int slot = nd % kKtDescRing;
+            const int type = __shfl_sync(0xffffffffu, desc[slot].type, 0);
+            dflags = __shfl_sync(0xffffffffu, desc[slot].flags, 0);
+            mbar_arrive_warp(&bars.desc_empty[slot]);
+            ++nd;
+            if (type == kKtChunk) have = true;
+            else if (type == kKtEnd) done = true;
         }
-        if (!wait(&bars.k_full[n % kKtKStages], (n / kKtKStages) & 1, kSiteKtMmaK, n)) break;
-        if (n >= 2 && !wait(&bars.p_full[n & 1], ((n - 2) >> 1) & 1, kSiteKtMmaP, n)) break;
-        tc_fence_after();
-        const uint32_t kst =
-            __shfl_sync(0xffffffffu, k_addr + (n % kKtKStages) * KtLayout::kKVBytes, 0);
-        const uint32_t tS = __shfl_sync(0xffffffffu, tmem + 64 * (n & 1), 0);
+        if (s_ready) {  // S^T[key, q] = K . Q^T for chunk ns
+            tc_fence_after();
+            if (dflags & kKtFirst) cur_o = qi++;
+            const int n = ns;
+            const uint32_t kst =
+                __shfl_sync(0xffffffffu, k_addr + (n % kKtKStages) * KtLayout::kKVBytes, 0);
+            const uint32_t tS = __shfl_sync(0xffffffffu, tmem + 64 * (n & 1), 0);
 #pragma unroll
-        for (int kk = 0; kk < kKtD / 16; ++kk) {
-            const int pn = kk >> 2, off = (kk & 3) * 32;
-            const uint64_t adesc = sw128_desc(kst + pn * KtLayout::kPanelKV + off, 16, 1024);
-            const uint64_t bdesc = sw128_desc(q_addr + pn * KtLayout::kPanelQ + off, 16, 1024);
-            mma_ss_warp(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kKtD / 16; ++kk) {
+                const int pn = kk >> 2, off = (kk & 3) * 32;
+                const uint64_t adesc = sw128_desc(kst + pn * KtLayout::kPanelKV + off, 16, 1024);
+                const uint64_t bdesc = sw128_desc(q_addr + pn * KtLayout::kPanelQ + off, 16, 1024);
+                mma_ss_warp(tS, adesc, bdesc, idS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit_warp(&bars.s_full[n & 1]);
+            mma_commit_warp(&bars.k_empty[n % kKtKStages]);
+            if (dflags & kKtLast) mma_commit_warp(bars.q_empty);
+            // bits 0-4 flags, 5 O^T buffer, 6 buffer used before, 7 (item / 2) % 2
+            const uint32_t info = (uint32_t)(dflags & 31) | ((uint32_t)(cur_o & 1) << 5) |
+                                  ((cur_o >= 2 ? 1u : 0u) << 6) | ((uint32_t)((cur_o >> 1) & 1) << 7);
+            pend = (pend & ~(0xFFu << ((n & 3) * 8))) | (info << ((n & 3) * 8));
+            ++ns;
+            have = false;
         }
-        mma_commit_warp(&bars.s_full[n & 1]);
-        mma_commit_warp(&bars.k_empty[n % kKtKStages]);
-        if (flags & kKtLast) mma_commit_warp(bars.q_empty);
-        mbar_arrive_warp(&bars.desc_empty[slot]);
-        issue_o();  // the previous chunk, while the softmax works on this one
-        pend = n;
-        pend_flags = flags;
-        pend_o = cur_o;
+        if (o_ready) {  // O^T[dim, q] += V^T . P^T for chunk no
+            tc_fence_after();
+            const int m = no;
+            const uint32_t vst =
+                __shfl_sync(0xffffffffu, v_addr + (m % kKtVStages) * KtLayout::kKVBytes, 0);
+            const uint32_t pst = __shfl_sync(0xffffffffu, p_addr + (m & 1) * KtLayout::kPBytes, 0);
+            const uint32_t tO = __shfl_sync(0xffffffffu, tmem + 128 + 64 * ((po >> 5) & 1), 0);
+            const uint32_t acc0 = __shfl_sync(0xffffffffu, (po & kKtFirst) ? 0u : 1u, 0);
+#pragma unroll
+            for (int kk = 0; kk < kKtKeys / 16; ++kk) {
+                // A = V^T (d x keys) stored MN-major: d-panels of 64 at kPanelKV apart,
+                // 16 keys = 16 rows of 128 bytes per K-step
+                const uint64_t adesc = sw128_desc(vst + kk * 2048, KtLayout::kPanelKV, 1024);
+                // B = P^T (64 queries x keys) stored MN-major: one 128-byte row per key
+                const uint64_t bdesc = sw128_desc(pst + kk * 2048, KtLayout::kPBytes, 1024);
+                mma_ss_warp(tO, adesc, bdesc, idO, kk == 0 ? acc0 : 1u);
+            }
+            mma_commit_warp(&bars.p_free[m & 1]);
+            mma_commit_warp(&bars.v_empty[m % kKtVStages]);
+            if (po & kKtLast) mma_commit_warp(&bars.o_full[(po >> 5) & 1]);
+            ++no;
+        }
     }
-    issue_o();
     if (!ok && lane == 0) kt_set_abort(abort, p.err, p.seq);
     // every MMA of this warp must have finished before TMEM is released
     mma_commit_warp(bars.drain);
@@ -568,8 +602,29 @@ __device__ void kt_run_softmax(const KtParams& p, uint8_t* sm, const KtBars& bar
 
     for (int nd = 0;; ++nd) {
         const int slot = nd % kKtDescRing;
+        // One probe across lanes for the three barriers a chunk normally waits
+        // on (its descriptor, its S^T, its P^T buffer free); those found
+        // complete cost no further wait.
+        bool pre_desc, pre_s, pre_pf;
+        {
+            uint64_t* bar = bars.q_full;
+            uint32_t par = 0;
+            bool live = false;
+            if (lane == 0) {
+                bar = &bars.desc_full[slot]; par = (nd / kKtDescRing) & 1; live = true;
+            } else if (lane == 1) {
+                bar = &bars.s_full[nc & 1]; par = (nc >> 1) & 1; live = true;
+            } else if (lane == 2 && nc >= 2) {
+                bar = &bars.p_free[nc & 1]; par = ((nc - 2) >> 1) & 1; live = true;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, live ? mbar_test_wait(bar, par) : true);
+            pre_desc = bal & 1u;
+            pre_s = (bal >> 1) & 1u;
+            pre_pf = (bal >> 2) & 1u;
+        }
         int type = kKtEnd, flags = 0, qh = 0, qb = 0;
-        if (wait(&bars.desc_full[slot], (nd / kKtDescRing) & 1, kSiteKtSoftmaxDesc, -1 - nd)) {
+        if (pre_desc ||
+            wait(&bars.desc_full[slot], (nd / kKtDescRing) & 1, kSiteKtSoftmaxDesc, -1 - nd)) {
             type = desc[slot].type;
             flags = desc[slot].flags;
             qh = desc[slot].qh;
@@ -596,23 +651,35 @@ __device__ void kt_run_softmax(const KtParams& p, uint8_t* sm, const KtBars& bar
         const bool valid = half == 0 || (flags & kKtHalf1);
         const bool diag = (half == 0 ? (flags & kKtDiag0) : (flags & kKtDiag1)) != 0;
 
-        // --- scores of this key for the warp's 32 queries (raw dot products)
+        // --- scores of this key for the warp's 32 queries (raw dot products).
+        // A warp's 32 keys lie in one half, so `valid` and `diag` are
+        // warp-uniform; only an unused half or the diagonal block needs the
+        // key's valid queries as a bit mask (applied branch-free: a divergent
+        // branch per element costs more than the whole loop).
         float v[32];
-        if (wait(&bars.s_full[b], (n >> 1) & 1, kSiteKtSoftmaxS, n)) {
+        if (pre_s || wait(&bars.s_full[b], (n >> 1) & 1, kSiteKtSoftmaxS, n)) {
             tc_fence_after();
             uint32_t r[32];
             tmem_ld32(tbase + 64 * b, r);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const bool keep = valid && (!diag || 32 * ch + i >= kk);
-                v[i] = keep ? __uint_as_float(r[i]) : -INFINITY;
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            if (!valid || diag) {
+                const int cut = kk - 32 * ch;  // first valid query of the diagonal block
+                const uint32_t vmask =
+                    !valid ? 0u : (cut <= 0 ? 0xffffffffu : (cut >= 32 ? 0u : ~0u << cut));
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = (vmask >> i) & 1u ? v[i] : -INFINITY;
             }
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = -INFINITY;
         }
-        // --- vote: does some score pass its query's reference by more than 2^8?
-        bool need = false;
+        // --- exponent arguments x = s c - M and the vote: does some score pass
+        // its query's reference by more than 2^8?  A query without a reference
+        // yet (-inf) counts as passing it.  Without a rescale (the usual case)
+        // these x are the exponents of P as they stand.
+        float x[32];
+        float xmax = -INFINITY;
         {
             const float4* m4 = reinterpret_cast<const float4*>(Mq + 32 * ch);
 #pragma unroll
@@ -621,11 +688,15 @@ __device__ void kt_run_softmax(const KtParams& p, uint8_t* sm, const KtBars& bar
                 const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float s = v[4 * j + u];
-                    need |= s > -INFINITY && (mv[u] == -INFINITY || s * cs - mv[u] > kKtRescale);
+                    const float mr = mv[u] == -INFINITY ? -3.0e38f : mv[u];
+                    x[4 * j + u] = fmaf(v[4 * j + u], cs, -mr);
                 }
             }
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                xmax = fmaxf(xmax, fmaxf(fmaxf(x[i], x[i + 1]), fmaxf(x[i + 2], x[i + 3])));
         }
+        const bool need = xmax > kKtRescale;
         const bool wneed = __any_sync(0xffffffffu, need);
         if (lane == 0) flags_sm[b * 8 + warp] = wneed ? 1 : 0;
         if (kt_softmax_bar(!ok || *abort)) break;
@@ -669,29 +740,30 @@ __device__ void kt_run_softmax(const KtParams& p, uint8_t* sm, const KtBars& bar
             }
         }
         // --- P^T = 2^(s c - M): the buffer is free once the O^T two chunks back has run
-        if (n >= 2) wait(&bars.p_free[b], ((n - 2) >> 1) & 1, kSiteKtSoftmaxO, n);
+        if (n >= 2 && !pre_pf) wait(&bars.p_free[b], ((n - 2) >> 1) & 1, kSiteKtSoftmaxO, n);
         if (ok) {
-            uint32_t pk[16];
-            const float4* m4 = reinterpret_cast<const float4*>(Mq + 32 * ch);
+            if (rescale) {  // the references moved: exponents against the new ones
+                const float4* m4 = reinterpret_cast<const float4*>(Mq + 32 * ch);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 mm = m4[j];
-                const float mu[4] = {mm.x == -INFINITY ? 0.f : mm.x, mm.y == -INFINITY ? 0.f : mm.y,
-                                     mm.z == -INFINITY ? 0.f : mm.z, mm.w == -INFINITY ? 0.f : mm.w};
+                for (int j = 0; j < 8; ++j) {
+                    const float4 mm = m4[j];
+                    const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
 #pragma unroll
-                for (int u = 0; u < 4; u += 2) {
-                    const int i = 4 * j + u;
-                    const uint64_t x2 = f2_fma(f2_pack(v[i], v[i + 1]), f2_pack(cs, cs),
-                                               f2_pack(-mu[u], -mu[u + 1]));
-                    float x0, x1;
-                    f2_unpack(x2, x0, x1);
-                    const uint64_t p2 = (j & 3) == 3 ? exp2_poly2(x2) : f2_pack(ex2(x0), ex2(x1));
-                    float p0, p1;
-                    f2_unpack(p2, p0, p1);
-                    l[i] += p0;
-                    l[i + 1] += p1;
-                    pk[i >> 1] = pack_bf16(p0, p1);
+                    for (int u = 0; u < 4; ++u)
+                        x[4 * j + u] =
+                            fmaf(v[4 * j + u], cs, -(mv[u] == -INFINITY ? 0.f : mv[u]));
                 }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const uint64_t x2 = f2_pack(x[i], x[i + 1]);
+                const uint64_t p2 = ((i >> 1) & 3) == 3 ? exp2_poly2(x2) : f2_pack(ex2(x[i]), ex2(x[i + 1]));
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
+                l[i] += p0;
+                l[i + 1] += p1;
+                pk[i >> 1] = pack_bf16(p0, p1);
             }
             // row kl of the 128-byte-swizzled P^T tile: 16-byte chunk c at c ^ (kl % 8)
             uint8_t* prow = pbuf + b * KtLayout::kPBytes + kl * 128;
