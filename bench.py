@@ -48,7 +48,7 @@ def log(msg):
 
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SOURCES = ["attn.cu", "attn_kt.cu", "softmax_math.cuh", "exp2_poly.h", "ptx.cuh", "internal.h"]
+ATTN_SOURCES = ["attn.cu", "softmax_math.cuh", "exp2_poly.h", "ptx.cuh", "internal.h"]
 
 
 def parse_args(argv=None):
@@ -66,6 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-1m", action="store_true",
                     help="skip the 1M-token layer measured after the main workload (at_1m)")
+    ap.add_argument("--bs-engine", default="row", choices=["row", "key"],
+                    help="engine for Block-Sparse heads (row-major tiles, or key-major)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0,
                     help="approximate CPU seconds for the oracle baseline sample")
     return ap.parse_args(argv)
@@ -457,6 +459,7 @@ def run_minfer(args):
     barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
     w = workload_of(args)
+    B.mi_set_bs_engine(B.BS_ENGINE_KEY if args.bs_engine == "key" else B.BS_ENGINE_ROW)
     log(f"generating {w.name} (N={w.N})")
     x = synth.make_inputs(w, device=str(dev))
     torch.cuda.synchronize()
@@ -592,7 +595,8 @@ def run_minfer(args):
             "metric": METRIC, "value": job_value(ms_step_max, world), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step_max,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_of(w),
+            "data": "synthetic",
+            "config": dict(config_of(w), **({"bs_engine": "key"} if args.bs_engine == "key" else {})),
             "ms_index": ms_index, "ms_prep": ms_prep, "ms_attn": ms_attn,
             "tile_density": tile_density(w, tiles),
             "gathered_column_blocks": cols,

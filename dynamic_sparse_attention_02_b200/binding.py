@@ -33,7 +33,7 @@ EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_by
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
            "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
            "mi_vs_index_static", "mi_dense_attn", "mi_prefill_workspace_bytes_heads",
-           "mi_prefill_layer_heads", "mi_debug_set_wait_budget"]
+           "mi_prefill_layer_heads", "mi_debug_set_wait_budget", "mi_set_bs_engine"]
 
 
 class MinferError(RuntimeError):
@@ -87,6 +87,7 @@ def _lib_handle():
         lib.mi_prefill_layer_heads.argtypes = [P, P, P, I, I, I, I, F, P, P, P, P, P, P, SZ, P,
                                                P]
         lib.mi_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
+        lib.mi_set_bs_engine.argtypes = [ctypes.c_int]
         for name in EXPORTS[5:]:
             if name != "mi_prefill_workspace_bytes_heads":
                 getattr(lib, name).restype = I
@@ -191,6 +192,16 @@ def mi_debug_set_wait_budget(cycles: int) -> None:
     """Clock budget of the kernels' abortable waits for later launches
     (<= 0: the default).  Failure-path tests only."""
     _check("mi_debug_set_wait_budget", _lib_handle().mi_debug_set_wait_budget(int(cycles)))
+
+
+BS_ENGINE_ROW = 0
+BS_ENGINE_KEY = 1
+
+
+def mi_set_bs_engine(engine: int) -> None:
+    """Engine for Block-Sparse heads in later launches: BS_ENGINE_ROW (the
+    default) or BS_ENGINE_KEY (key-major tiles, d = 128)."""
+    _check("mi_set_bs_engine", _lib_handle().mi_set_bs_engine(int(engine)))
 
 
 def mi_status_str(status: int) -> str:

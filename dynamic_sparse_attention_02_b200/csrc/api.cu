@@ -15,6 +15,7 @@ using namespace minfer;
 namespace {
 thread_local int g_last_cuda_error = 0;
 std::atomic<long long> g_wait_budget{0};  // 0: the default bound
+std::atomic<int> g_bs_engine{MI_BS_ENGINE_ROW};
 }  // namespace
 
 long long minfer::wait_budget_cycles() {
@@ -31,6 +32,12 @@ int minfer::cuda_status(cudaError_t e) {
 }
 
 namespace {
+
+// Block-Sparse heads go to the key-major engine only when it is selected and
+// serves the launch's shapes.
+bool use_key_major(const AttnLaunch& a) {
+    return g_bs_engine.load() == MI_BS_ENGINE_KEY && kt_attn_supported(a);
+}
 
 // Shapes every entry point shares.  Fills `hl` with the listed heads
 // (pattern and per-pattern position filled by the caller).
@@ -280,7 +287,7 @@ int mi_block_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, i
     a.blk_cnt = blk_cnt;
     a.topk = topk;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return cuda_status(kt_attn_supported(a) ? launch_kt_attn(a, st) : launch_sparse_attn(a, st));
+    return cuda_status(use_key_major(a) ? launch_kt_attn(a, st) : launch_sparse_attn(a, st));
 }
 
 int mi_ashape_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N,
@@ -447,9 +454,9 @@ int prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, 
     a.sink_h = lp.sink_h;
     a.window_h = lp.win_h;
     a.n_asw = lp.n_a;
-    // Block-Sparse heads run on the key-major engine where it applies, the
-    // rest (and all heads otherwise) in one launch of the row-major engine
-    if (lp.bs.n && kt_attn_supported(a)) {
+    // With the key-major engine selected, Block-Sparse heads run on it where
+    // it applies; the rest (all heads otherwise) in one row-major launch
+    if (lp.bs.n && use_key_major(a)) {
         AttnLaunch abs = a;
         abs.heads.n = 0;
         a.heads.n = 0;
@@ -492,6 +499,12 @@ int mi_prefill_layer_heads(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v,
                            void* const* stage_events) {
     return prefill_layer(q, k, v, Hq, Hkv, N, d, scale, pattern, params, true, out, lse,
                          err_count, ws, ws_bytes, stream, stage_events);
+}
+
+int mi_set_bs_engine(int engine) {
+    if (engine != MI_BS_ENGINE_ROW && engine != MI_BS_ENGINE_KEY) return MI_ERR_INVALID_ARG;
+    g_bs_engine.store(engine);
+    return MI_OK;
 }
 
 int mi_debug_set_wait_budget(long long cycles) {

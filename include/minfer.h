@@ -306,6 +306,25 @@ int mi_debug_wait_failure(int32_t* record8);
  */
 int mi_debug_set_wait_budget(long long cycles);
 
+/*
+ * Engine for Block-Sparse heads in the launches that follow (process-wide):
+ *   MI_BS_ENGINE_ROW (0, the default) -- the row-major engine every pattern
+ *     uses: 128 query rows per tensor-core tile (two 64-row query blocks),
+ *     each 64-key chunk the union of the two blocks' chosen blocks;
+ *   MI_BS_ENGINE_KEY (1) -- the key-major engine for d = 128: one 64-row
+ *     query block per work item, two of ITS chosen key blocks per 128-key
+ *     tile (S^T = K Q^T, O^T += V^T P^T), so no computed score is unused.
+ * Both follow the Block-Sparse definition of MInference 1.0 (aifetchly
+ * guide, "3. The Block-Sparse Pattern") and give the same results up to
+ * rounding order.  The row-major engine is the faster one on the Block-Sparse
+ * workloads measured so far; the key-major one is kept for comparison.
+ * Returns MI_ERR_INVALID_ARG for any other value.  Not thread-safe against
+ * concurrent launches.
+ */
+#define MI_BS_ENGINE_ROW 0
+#define MI_BS_ENGINE_KEY 1
+int mi_set_bs_engine(int engine);
+
 #ifdef __cplusplus
 }
 #endif

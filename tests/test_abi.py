@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = header_functions()
-    assert len(names) == 17
+    assert len(names) == 18
     assert sorted(B.EXPORTS) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -40,6 +40,13 @@ def test_status_strings(lib):
         assert B.mi_status_str(code)
     assert B.mi_status_str(99) == "unknown status"
     assert "sm_100a" in B.mi_version()
+
+
+def test_bs_engine_selector(lib):
+    assert lib.mi_set_bs_engine(2) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_set_bs_engine(-1) == B.MI_ERR_INVALID_ARG
+    assert lib.mi_set_bs_engine(B.BS_ENGINE_KEY) == B.MI_OK
+    assert lib.mi_set_bs_engine(B.BS_ENGINE_ROW) == B.MI_OK
 
 
 FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation runs first

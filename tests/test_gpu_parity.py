@@ -26,6 +26,14 @@ def _built():
     build.build()
 
 
+@pytest.fixture(params=[B.BS_ENGINE_ROW, B.BS_ENGINE_KEY], ids=["row", "key"])
+def bs_engine(request):
+    """Each Block-Sparse attention case runs on both engines."""
+    B.mi_set_bs_engine(request.param)
+    yield request.param
+    B.mi_set_bs_engine(B.BS_ENGINE_ROW)
+
+
 # ------------------------------------------------------------ VS index
 
 @pytest.mark.parametrize("Hq,Hkv,N,d,L,kv,ks", [
@@ -128,7 +136,7 @@ def test_ashape_attn_matches_oracle(Hq, Hkv, N, d, sink, window):
     (4, 1, 1024, 128, 4), (2, 2, 576, 64, 3), (2, 1, 2048, 128, 100),
     (6, 2, 4096, 128, 9),    # more items than one CTA per SM takes at once, odd topk
     (1, 1, 64, 128, 1)])     # a single query block
-def test_block_sparse_attn_matches_oracle(Hq, Hkv, N, d, topk):
+def test_block_sparse_attn_matches_oracle(Hq, Hkv, N, d, topk, bs_engine):
     q, k, v = rand_bf16(Hq, Hkv, N, d, 12)
     nB = N // 64
     bi = np.full((Hq, nB, topk), -1, np.int32)
@@ -145,7 +153,7 @@ def test_block_sparse_attn_matches_oracle(Hq, Hkv, N, d, topk):
         check_attn(out[h], lse[h], *refs[h], what=f"bs h{h}")
 
 
-def test_block_sparse_attn_unusual_lists_and_empty_rows():
+def test_block_sparse_attn_unusual_lists_and_empty_rows(bs_engine):
     """Block lists as a caller may pass them: unsorted, with duplicates, -1
     padding in the middle, entries past the query block or outside [0, N/64)
     (skipped and counted), counts above topk (clamped to topk) and rows with no
@@ -191,7 +199,7 @@ def test_block_sparse_attn_unusual_lists_and_empty_rows():
     assert (out[0, 192:256] == 0).all() and torch.isneginf(lse[0, 192:256]).all()
 
 
-def test_block_sparse_attn_rescales_mid_item():
+def test_block_sparse_attn_rescales_mid_item(bs_engine):
     """A query block whose later key blocks score far above its first ones:
     the per-query reference max must move up mid-item (the lazy rescale of
     O and of the running sums), and a block scoring far below must not."""
@@ -328,7 +336,7 @@ def test_full_budgets_equal_dense_sdpa():
 
 
 @pytest.mark.parametrize("N,d,L", [(1024, 128, 64), (576, 64, 64), (2560, 128, 100)])
-def test_prefill_layer_mixed_matches_oracle(N, d, L):
+def test_prefill_layer_mixed_matches_oracle(N, d, L, bs_engine):
     """The pattern router: mixed A-shape / VS / BS / dense heads in one launch
     (last_q = 100: the VS index merges two 64-row groups per head)."""
     w = synth.workload("mixed_n256k_llama3_8b", Hq=8, Hkv=2, N=N, d=d)

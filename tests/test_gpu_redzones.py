@@ -134,7 +134,7 @@ def _attn_call(which, q, k, v, heads, out, lse, ws):
                           device="cuda")
         si = torch.tensor([[0, 64, 200, -1]] * len(heads), dtype=torch.int32, device="cuda")
         B.mi_vs_sparse_attn(q, k, v, vi, si, heads=heads, out=out, lse=lse, ws=ws)
-    elif which == "bs":
+    elif which in ("bs", "bs_key"):
         nB = N // 64
         bi = torch.full((len(heads), nB, 3), -1, dtype=torch.int32, device="cuda")
         for bq in range(nB):
@@ -142,14 +142,18 @@ def _attn_call(which, q, k, v, heads, out, lse, ws):
             bi[:, bq, 1] = 0
         bc = torch.full((len(heads), nB), 2, dtype=torch.int32, device="cuda")
         bc[:, 0] = 1
-        B.mi_block_sparse_attn(q, k, v, bi, bc, heads=heads, out=out, lse=lse)
+        B.mi_set_bs_engine(B.BS_ENGINE_KEY if which == "bs_key" else B.BS_ENGINE_ROW)
+        try:
+            B.mi_block_sparse_attn(q, k, v, bi, bc, heads=heads, out=out, lse=lse)
+        finally:
+            B.mi_set_bs_engine(B.BS_ENGINE_ROW)
     elif which == "ashape":
         B.mi_ashape_attn(q, k, v, 64, 128, heads=heads, out=out, lse=lse)
     else:
         B.mi_dense_attn(q, k, v, heads=heads, out=out, lse=lse)
 
 
-@pytest.mark.parametrize("which", ["vs", "bs", "ashape", "dense"])
+@pytest.mark.parametrize("which", ["vs", "bs", "bs_key", "ashape", "dense"])
 def test_attention_touches_listed_heads_only(which):
     Hq, Hkv, N, d = 6, 2, 640, 128
     q, k, v = rand_bf16(Hq, Hkv, N, d, 43)
