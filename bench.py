@@ -66,6 +66,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-1m", action="store_true",
                     help="skip the 1M-token layer measured after the main workload (at_1m)")
+    ap.add_argument("--no-1m-ranges", action="store_true",
+                    help="skip the 1M layer with range slash tiles (at_1m.slash_ranges)")
+    ap.add_argument("--slash-tiles", default="blocks", choices=["blocks", "ranges"],
+                    help="how VS heads of the main workload read their diagonals")
     ap.add_argument("--bs-engine", default="row", choices=["row", "key"],
                     help="engine for Block-Sparse heads (row-major tiles, or key-major)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0,
@@ -83,9 +87,10 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def params_of(w, B):
+def params_of(w, B, ranges=False):
     return B.make_params(last_q=w.last_q, vertical_size=w.vertical_size, slash_size=w.slash_size,
-                         topk_blocks=w.topk_blocks, sink=w.sink, window=w.window)
+                         topk_blocks=w.topk_blocks, sink=w.sink, window=w.window,
+                         slash_tiles=B.MI_SLASH_RANGES if ranges else B.MI_SLASH_BLOCKS)
 
 
 def attn_source_sha():
@@ -198,6 +203,48 @@ def vs_useful_flops(v_idx, s_idx, N, d):
     cnt_le = np.cumsum(D)  # |{delta in D : delta <= x}|
     bj = V // 64
     cols = int(np.sum((nB - bj) - cnt_le[nB - 1 - bj]))
+    return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
+
+
+def vs_range_useful_flops(v_idx, s_idx, N, d):
+    """Useful FLOPs of one VS head whose diagonals are read as ranges: query
+    block bq takes key u iff some selected o has 64 bq - u <= o <= 64 bq - u + 63,
+    i.e. R[64 bq - u] with R[x] = "a selected offset in [x, x + 63]" (x >= -63).
+    Per query block, the kept keys form runs of R; each run of length n costs
+    ceil(n / 64) 64-key tiles of 64 rows.  Gathered columns: those outside the
+    block's runs, 64 rows each.  Returns (flops, 64x64-equivalent tiles,
+    gathered column-blocks)."""
+    nB = N // 64
+    s = np.unique(s_idx[(s_idx >= 0) & (s_idx < N)])
+    S = np.zeros(N + 64, np.int64)
+    S[s] = 1
+    cs = np.concatenate([[0], np.cumsum(S)])
+    x = np.arange(-63, N)                              # R over x in [-63, N)
+    lo, hi = np.clip(x, 0, N), np.clip(x + 63, -1, N - 1)
+    R = (cs[hi + 1] - cs[lo]) > 0
+    # runs of R, then per query block bq the windows of the runs clipped to x <= 64 bq
+    m = np.concatenate([[0], R.astype(np.int8), [0]])
+    dm = np.diff(m)
+    rs = np.nonzero(dm == 1)[0] - 63                   # run starts (x coordinates)
+    re = np.nonzero(dm == -1)[0] - 1 - 63              # run ends, inclusive
+    full = (re - rs + 64) // 64
+    cf = np.concatenate([[0], np.cumsum(full)])
+    lim = 64 * np.arange(nB)
+    j = np.searchsorted(re, lim, side="right")         # runs ending at or before lim
+    win = cf[j]
+    jj = np.minimum(j, max(len(rs) - 1, 0))
+    part = (j < len(rs)) & (rs[jj] <= lim) if len(rs) else np.zeros(nB, bool)
+    win = win + np.where(part, (lim - rs[jj] + 64) // 64, 0) if len(rs) else win
+    tiles = int(win.sum())
+    # column c is kept by blocks bq >= c // 64; covered there iff R[64 bq - c], i.e. entry
+    # 64 (bq - c // 64) + 63 - c % 64 of R (which starts at x = -63): a stride-64 count
+    V = np.unique(v_idx[(v_idx >= 0) & (v_idx < N)])
+    Rp = np.zeros(64 * (nB + 1), np.int64)
+    Rp[:R.size] = R
+    C = np.cumsum(Rp.reshape(nB + 1, 64), axis=0)
+    cb, cl = V // 64, V % 64
+    covered = C[nB - 1 - cb, 63 - cl]
+    cols = int(np.sum((nB - cb) - covered))
     return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
 
 
@@ -383,9 +430,10 @@ def time_layer(B, w, x, params, ws, out, steps, warmup, ranks, dev):
     return ms_step, ms_index, ms_prep, ms_attn, clk
 
 
-def useful_work(B, w, x):
+def useful_work(B, w, x, ranges=False):
     """Algorithmic work of the layer's attention launch, from its own index:
-    (computed-tile FLOPs, 64x64 tiles, gathered column-blocks)."""
+    (computed-tile FLOPs, 64x64 tiles, gathered column-blocks); ranges: the
+    VS heads read their diagonals as 64-key ranges."""
     useful, tiles, cols = 0.0, 0, 0
     q, k, pat = x["q"], x["k"], np.asarray(x["pattern"])
     vs_heads = [h for h in range(w.Hq) if pat[h] == synth.PATTERN_VS]
@@ -396,7 +444,8 @@ def useful_work(B, w, x):
                                      heads=vs_heads)
         vi, si = v_idx.cpu().numpy(), s_idx.cpu().numpy()
         for i in range(len(vs_heads)):
-            f, t, c = vs_useful_flops(vi[i], si[i], w.N, w.d)
+            f, t, c = (vs_range_useful_flops if ranges else vs_useful_flops)(vi[i], si[i], w.N,
+                                                                              w.d)
             useful += f
             tiles += t
             cols += c
@@ -416,7 +465,7 @@ def tile_density(w, tiles):
     return tiles / (w.Hq * (w.N // 64) * (w.N // 64 + 1) / 2) if tiles else None
 
 
-def measure_1m(B, ranks, dev, peak):
+def measure_1m(B, ranks, dev, peak, with_ranges=True):
     """The metric's 1M half, measured in the same run: the 1M-token
     Vertical-Slash layer (32 query heads, 8 KV heads, d = 128, last_q 64,
     vertical 1000, slash 6096), 1 warm-up + 2 timed steps, with its own clock
@@ -426,26 +475,36 @@ def measure_1m(B, ranks, dev, peak):
     log(f"generating {w.name} (N={w.N})")
     x = synth.make_inputs(w, device=str(dev))
     torch.cuda.synchronize()
-    params = params_of(w, B)
-    ws = torch.empty(B.mi_prefill_workspace_bytes(w.Hq, w.Hkv, w.N, w.d, x["pattern"], params),
-                     dtype=torch.uint8, device=dev)
     out = torch.empty_like(x["q"])
     steps, warmup = 2, 1
-    ms_step, ms_index, ms_prep, ms_attn, clk = time_layer(B, w, x, params, ws, out, steps,
-                                                          warmup, ranks, dev)
-    useful, tiles, cols = useful_work(B, w, x)
-    eff = useful / (ms_attn * 1e-3) / 1e12
-    mhz = clk.get("sm_mhz")
-    rec = {"workload": w.name, "N": w.N, "steps": steps, "warmup": warmup,
-           "ms_per_layer": ms_step, "ms_index": ms_index, "ms_prep": ms_prep,
-           "ms_attn": ms_attn, "eff_tflops": eff, "frac_of_peak": eff / peak,
-           "flops_per_launch": useful, "tile_density": tile_density(w, tiles),
-           "gathered_column_blocks": cols,
-           "attn_kcycles": ms_attn * mhz if mhz else None,
-           "tensor_pipe": recorded_tensor_pipe(w.name),
-           # VS index (2 score passes, row merge, top-k), prep, attention
-           "gpu_launches": 6 * steps, "clocks": clk}
-    del x, ws, out
+
+    def leg(ranges):
+        params = params_of(w, B, ranges)
+        ws = torch.empty(B.mi_prefill_workspace_bytes(w.Hq, w.Hkv, w.N, w.d, x["pattern"],
+                                                      params), dtype=torch.uint8, device=dev)
+        ms_step, ms_index, ms_prep, ms_attn, clk = time_layer(B, w, x, params, ws, out, steps,
+                                                              warmup, ranks, dev)
+        del ws
+        useful, tiles, cols = useful_work(B, w, x, ranges)
+        eff = useful / (ms_attn * 1e-3) / 1e12
+        mhz = clk.get("sm_mhz")
+        return {"ms_per_layer": ms_step, "ms_index": ms_index, "ms_prep": ms_prep,
+                "ms_attn": ms_attn, "eff_tflops": eff, "frac_of_peak": eff / peak,
+                "flops_per_launch": useful, "tile_density": tile_density(w, tiles),
+                "gathered_column_blocks": cols,
+                "attn_kcycles": ms_attn * mhz if mhz else None, "clocks": clk}
+
+    rec = {"workload": w.name, "N": w.N, "steps": steps, "warmup": warmup}
+    rec.update(leg(False))
+    rec["tensor_pipe"] = recorded_tensor_pipe(w.name)
+    # VS index (2 score passes, row merge, top-k), prep, attention
+    rec["gpu_launches"] = 6 * steps
+    if with_ranges:
+        # the same layer with every diagonal read as 64-key ranges (MI_SLASH_RANGES):
+        # a different, sparser mask, so its time is not the metric's
+        log("1M layer with range slash tiles")
+        rec["slash_ranges"] = leg(True)
+    del x, out
     torch.cuda.empty_cache()
     return rec
 
@@ -465,7 +524,8 @@ def run_minfer(args):
     torch.cuda.synchronize()
     q, k, v = x["q"], x["k"], x["v"]
     pattern = x["pattern"]
-    params = params_of(w, B)
+    ranges = args.slash_tiles == "ranges"
+    params = params_of(w, B, ranges)
     ws = torch.empty(B.mi_prefill_workspace_bytes(w.Hq, w.Hkv, w.N, w.d, pattern, params),
                      dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
@@ -564,7 +624,7 @@ def run_minfer(args):
                  "tflops": 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq / (ms_dense * 1e-3) / 1e12}
         del dout
 
-    useful, tiles, cols = useful_work(B, w, x)
+    useful, tiles, cols = useful_work(B, w, x, ranges)
     dense_eq = 4.0 * w.d * w.N * (w.N + 1) / 2 * w.Hq
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -579,7 +639,7 @@ def run_minfer(args):
         x = {"q": q[0:1].cpu(), "k": k[0:1].cpu(), "v": v[0:1].cpu(), "pattern": pattern}
         del q, k, v, ws, out
         torch.cuda.empty_cache()
-        at_1m = measure_1m(B, ranks, dev, peak)
+        at_1m = measure_1m(B, ranks, dev, peak, with_ranges=not args.no_1m_ranges)
 
     line = None
     if rank == 0:
@@ -596,7 +656,8 @@ def run_minfer(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step_max,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": dict(config_of(w), **({"bs_engine": "key"} if args.bs_engine == "key" else {})),
+            "config": dict(config_of(w), **({"bs_engine": "key"} if args.bs_engine == "key" else {}),
+                           **({"slash_tiles": "ranges"} if ranges else {})),
             "ms_index": ms_index, "ms_prep": ms_prep, "ms_attn": ms_attn,
             "tile_density": tile_density(w, tiles),
             "gathered_column_blocks": cols,

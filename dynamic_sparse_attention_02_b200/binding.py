@@ -31,7 +31,8 @@ MI_BLOCK = 64
 # every symbol include/minfer.h declares
 EXPORTS = ["mi_status_str", "mi_last_cuda_error", "mi_version", "mi_workspace_bytes",
            "mi_prefill_workspace_bytes", "mi_vs_index", "mi_bs_index", "mi_vs_sparse_attn",
-           "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer", "mi_debug_wait_failure",
+           "mi_vs_range_attn", "mi_block_sparse_attn", "mi_ashape_attn", "mi_prefill_layer",
+           "mi_debug_wait_failure",
            "mi_vs_index_static", "mi_dense_attn", "mi_prefill_workspace_bytes_heads",
            "mi_prefill_layer_heads", "mi_debug_set_wait_budget", "mi_set_bs_engine"]
 
@@ -48,7 +49,7 @@ class MinferError(RuntimeError):
 class mi_params(ctypes.Structure):
     _fields_ = [("last_q", ctypes.c_int), ("vertical_size", ctypes.c_int),
                 ("slash_size", ctypes.c_int), ("topk_blocks", ctypes.c_int),
-                ("sink", ctypes.c_int), ("window", ctypes.c_int)]
+                ("sink", ctypes.c_int), ("window", ctypes.c_int), ("slash_tiles", ctypes.c_int)]
 
 
 _lib = None
@@ -74,6 +75,7 @@ def _lib_handle():
         lib.mi_bs_index.argtypes = [P, P, I, I, I, I, F, I, I, P, I, P, P, P, SZ, P]
         lib.mi_vs_sparse_attn.argtypes = [P, P, P, I, I, I, I, F, P, I, P, I, P, I, P, P, P, P,
                                           SZ, P]
+        lib.mi_vs_range_attn.argtypes = lib.mi_vs_sparse_attn.argtypes
         lib.mi_block_sparse_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, I, I, P, I, P, P, P,
                                              P, SZ, P]
         lib.mi_ashape_attn.argtypes = [P, P, P, I, I, I, I, F, I, I, P, I, P, P, P, P, SZ, P]
@@ -218,9 +220,13 @@ def mi_workspace_bytes(op, Hq, Hkv, N, d, n_heads=0, last_q=0, vertical_size=0, 
                                                 vertical_size, slash_size, topk_blocks))
 
 
+MI_SLASH_BLOCKS = 0
+MI_SLASH_RANGES = 1
+
+
 def make_params(last_q=64, vertical_size=1000, slash_size=6096, topk_blocks=100, sink=64,
-                window=1024) -> mi_params:
-    return mi_params(last_q, vertical_size, slash_size, topk_blocks, sink, window)
+                window=1024, slash_tiles=MI_SLASH_BLOCKS) -> mi_params:
+    return mi_params(last_q, vertical_size, slash_size, topk_blocks, sink, window, slash_tiles)
 
 
 def mi_prefill_workspace_bytes(Hq, Hkv, N, d, pattern, params: mi_params) -> int:
@@ -327,7 +333,9 @@ def _index_rows(name, t, n, q):
 
 
 def mi_vs_sparse_attn(q, k, v, v_idx, s_idx, heads=None, scale=0.0, out=None, lse=None,
-                      want_lse=True, err_count=None, ws=None, stream=None):
+                      want_lse=True, err_count=None, ws=None, stream=None, ranges=False):
+    """Vertical-Slash attention; ranges=True reads each diagonal as one
+    unaligned 64-key range per query block (mi_vs_range_attn)."""
     Hq, Hkv, N, d = _shape(q, k, v)
     harr, n, hp = _heads(heads, Hq)
     kv = _index_rows("v_idx", v_idx, n, q)
@@ -335,11 +343,12 @@ def mi_vs_sparse_attn(q, k, v, v_idx, s_idx, heads=None, scale=0.0, out=None, ls
     out, lse = _attn_out(q, out, lse, want_lse, err_count)
     ws, ws_bytes = _workspace(mi_workspace_bytes(MI_OP_VS_ATTN, Hq, Hkv, N, d, n, 0, kv, ks),
                               q.device, ws)
-    rc = _lib_handle().mi_vs_sparse_attn(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
-                                         _ptr(v_idx), kv, _ptr(s_idx), ks, hp, n, _ptr(out),
-                                         _ptr(lse), _ptr(err_count), _ptr(ws), ws_bytes,
-                                         _stream(stream))
-    _check("mi_vs_sparse_attn", rc)
+    name = "mi_vs_range_attn" if ranges else "mi_vs_sparse_attn"
+    rc = getattr(_lib_handle(), name)(_ptr(q), _ptr(k), _ptr(v), Hq, Hkv, N, d, scale,
+                                      _ptr(v_idx), kv, _ptr(s_idx), ks, hp, n, _ptr(out),
+                                      _ptr(lse), _ptr(err_count), _ptr(ws), ws_bytes,
+                                      _stream(stream))
+    _check(name, rc)
     return out, lse
 
 

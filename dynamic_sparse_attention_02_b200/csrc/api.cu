@@ -235,11 +235,16 @@ static void attn_common(AttnLaunch& a, const mi_bf16* q, const mi_bf16* k, const
     a.err_count = err_count;
 }
 
-int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
-                      int N, int d, float scale, const int32_t* v_idx, int vertical_size,
-                      const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
-                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
-                      void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Vertical-Slash attention with the diagonals read as 64x64 tiles or, with
+// `ranges`, as unaligned 64-key ranges.
+int vs_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv, int N, int d,
+            float scale, const int32_t* v_idx, int vertical_size, const int32_t* s_idx,
+            int slash_size, const int32_t* heads, int n_heads, mi_bf16* out, float* lse,
+            int32_t* err_count, void* ws, size_t ws_bytes, void* stream, bool ranges) {
     HeadList hl;
     int rc = check_shapes(q, k, Hq, Hkv, N, d, heads, n_heads, hl);
     if (rc) return rc;
@@ -253,17 +258,41 @@ int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int 
     VsPrepWs prep = carve_vs_prep(c, hl.n, N, kv);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = cuda_status(launch_vs_prep(v_idx, vertical_size, vertical_size, s_idx, slash_size,
-                                    slash_size, N, hl.n, prep, err_count, st));
+                                    slash_size, N, hl.n, prep, err_count, st, ranges));
     if (rc) return rc;
     AttnLaunch a;
     attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
     set_pattern(hl, MI_PATTERN_VS);
+    for (int i = 0; i < hl.n; ++i) hl.e[i] = with_ranges(hl.e[i], ranges);
     a.heads = hl;
     a.dbits = prep.dbits;
+    a.rwords = prep.rwords;
     a.vlist = prep.vlist;
     a.vcnt = prep.vcnt;
     a.vcap = prep.vcap;
     return cuda_status(launch_sparse_attn(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                      int N, int d, float scale, const int32_t* v_idx, int vertical_size,
+                      const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
+                      mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                      void* stream) {
+    return vs_attn(q, k, v, Hq, Hkv, N, d, scale, v_idx, vertical_size, s_idx, slash_size, heads,
+                   n_heads, out, lse, err_count, ws, ws_bytes, stream, false);
+}
+
+int mi_vs_range_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                     int N, int d, float scale, const int32_t* v_idx, int vertical_size,
+                     const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
+                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                     void* stream) {
+    return vs_attn(q, k, v, Hq, Hkv, N, d, scale, v_idx, vertical_size, s_idx, slash_size, heads,
+                   n_heads, out, lse, err_count, ws, ws_bytes, stream, true);
 }
 
 int mi_block_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
@@ -335,6 +364,7 @@ namespace {
 struct LayerPlan {
     HeadList all, vs, bs;
     int n_a = 0;
+    bool any_ranges = false;  // some VS head reads its diagonals as ranges
     mi_params pp{};  // layer-wide maxima: buffer sizes and index row strides
     int32_t kv_h[MI_MAX_HEADS], ks_h[MI_MAX_HEADS], tk_h[MI_MAX_HEADS];
     int32_t sink_h[MI_MAX_HEADS], win_h[MI_MAX_HEADS];
@@ -344,6 +374,7 @@ int plan_layer(int Hq, int N, const int8_t* pattern, const mi_params* params, bo
                LayerPlan& lp) {
     lp.vs.n = lp.bs.n = 0;
     lp.n_a = 0;
+    lp.any_ranges = false;
     int L = -1, kv_max = 0, ks_max = 0, tk_max = 0;
     for (int h = 0; h < Hq; ++h) {
         const mi_params& ph = params[per_head ? h : 0];
@@ -366,7 +397,11 @@ int plan_layer(int Hq, int N, const int8_t* pattern, const mi_params* params, bo
                 lp.ks_h[lp.vs.n] = ks;
                 kv_max = kv > kv_max ? kv : kv_max;
                 ks_max = ks > ks_max ? ks : ks_max;
-                lp.all.e[h] = pack_head(h, MI_PATTERN_VS, lp.vs.n);
+                if (ph.slash_tiles != MI_SLASH_BLOCKS && ph.slash_tiles != MI_SLASH_RANGES)
+                    return MI_ERR_INVALID_ARG;
+                const bool rg = ph.slash_tiles == MI_SLASH_RANGES;
+                lp.any_ranges |= rg;
+                lp.all.e[h] = with_ranges(pack_head(h, MI_PATTERN_VS, lp.vs.n), rg);
                 lp.vs.e[lp.vs.n] = pack_head(h, MI_PATTERN_VS, lp.vs.n);
                 ++lp.vs.n;
                 break;
@@ -435,7 +470,7 @@ int prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, 
     if (lp.vs.n) {
         rc = cuda_status(launch_vs_prep(w.v_idx, pp.vertical_size, pp.vertical_size, w.s_idx,
                                         pp.slash_size, pp.slash_size, N, lp.vs.n, w.prep,
-                                        err_count, st));
+                                        err_count, st, lp.any_ranges));
         if (rc) return rc;
     }
     if ((rc = rec(MI_STAGE_PREP_DONE))) return rc;
@@ -443,6 +478,7 @@ int prefill_layer(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, 
     attn_common(a, q, k, v, Hq, Hkv, N, d, scale, out, lse, err_count);
     a.heads = lp.all;
     a.dbits = w.prep.dbits;
+    a.rwords = w.prep.rwords;
     a.vlist = w.prep.vlist;
     a.vcnt = w.prep.vcnt;
     a.vcap = w.prep.vcap;

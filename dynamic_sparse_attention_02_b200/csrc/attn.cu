@@ -63,7 +63,7 @@ constexpr int kKVPanel = kChunkKeys * 128;  // 64 rows x one panel
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by >8
 
-enum : int { kChunkNone = 0, kChunkBlock = 1, kChunkGather = 2 };
+enum : int { kChunkNone = 0, kChunkBlock = 1, kChunkGather = 2, kChunkRange = 3 };
 // info flag: every row of the super tile takes every key of the chunk (a block
 // below the diagonal that all four query blocks take, outside A-shape)
 constexpr int kChunkWhole = 1 << 9;
@@ -71,9 +71,9 @@ constexpr int kChunkWhole = 1 << 9;
 struct ChunkDesc {
     int info;  // type | need << 4 | last << 8 | whole << 9 (see kChunkWhole)
     int type, last, need, ncols;
-    int b, m;  // block chunks: key block and its 4-bit query-block mask
+    int b, m;  // block chunks: key block and its 4-bit query-block mask; ranges: first key
     int cols[kChunkKeys];      // gathers: the columns, ascending
-    uint64_t qmask[4];         // gathers: per query block, the columns it takes
+    uint64_t qmask[4];         // gathers and ranges: per query block, the keys it takes
 };
 
 struct GatherHeld {
@@ -120,6 +120,7 @@ struct AttnParams {
     int Hq, Hkv, N, nB, n_super;
     float scale_log2;
     const uint32_t* dbits;
+    const uint64_t* rwords;
     int nBw;
     const int32_t* vlist;
     const int32_t* vcnt;
@@ -294,6 +295,46 @@ struct Producer {
         ++nkv;
     }
 
+    // 64 consecutive keys from key c0 (any offset; TMA rows past the KV head's
+    // end are another head's or zero fill, and no query block takes them) with
+    // the keys each query block takes
+    __device__ void window(int c0, const uint64_t (&qm)[4]) {
+        if (!ok) return;
+        probe_next();
+        ChunkDesc* d = acquire_desc();
+        if (!d) return;
+        if (lane == 0) {
+            const int need = (qm[0] | qm[1] ? 1 : 0) | (qm[2] | qm[3] ? 2 : 0);
+            d->info = kChunkRange | (need << 4);
+            d->type = kChunkRange;
+            d->last = 0;
+            d->need = need;
+            d->ncols = 0;
+            d->b = c0;
+            d->m = 0;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) d->qmask[qq] = qm[qq];
+        }
+        publish_desc();
+        int st;
+        if (!acquire_kv(st)) return;
+        if (lane == 0) {
+            const int row = g * p.N + c0;
+            mbar_arrive_expect_tx(&bars.kv_full[st], 2 * L::kKVBytes);
+            uint8_t* kd = sm + L::k_off + st * L::kKVBytes;
+            uint8_t* vd = sm + L::v_off + st * L::kKVBytes;
+            const uint64_t pol = l2_policy_evict_last();
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_2d_hint(kd + pn * kKVPanel, tmK, 64 * pn, row, &bars.kv_full[st], pol);
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_2d_hint(vd + pn * kKVPanel, tmV, 64 * pn, row, &bars.kv_full[st], pol);
+        }
+        __syncwarp();
+        ++nkv;
+    }
+
     // up to 64 gathered columns
     __device__ void gather(int n) {
         if (!ok) return;
@@ -385,6 +426,9 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
     const int lane = threadIdx.x & 31;
     const uint32_t e = p.heads.e[pos];
     const int qh = head_qh(e), pattern = head_pattern(e), pidx = head_pidx(e);
+    // Vertical-Slash head whose diagonals select unaligned 64-key ranges
+    const bool ranges = pattern == MI_PATTERN_VS && head_ranges(e);
+    const uint64_t* rw = ranges ? p.rwords + (size_t)pidx * p.nB : nullptr;
     const int g = kv_head_of(qh, p.Hq, p.Hkv);
     const int qb0 = 4 * T;
     const int nqb = min(4, p.nB - qb0);
@@ -403,7 +447,7 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
     }
 
     // per-pattern block map
-    if (pattern == MI_PATTERN_VS) {
+    if (pattern == MI_PATTERN_VS && !ranges) {
         const uint32_t* src = p.dbits + (size_t)pidx * p.nBw;
         for (int w = lane; w < p.nBw; w += 32) patmap[w] = src[w];
     } else if (pattern == MI_PATTERN_BS) {
@@ -432,8 +476,52 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
                    reinterpret_cast<GatherHeld*>(sm + L::held_off), g};
     pr.lane = lane;
 
+    // --- ranges: the keys the super tile's query blocks take, as 64-key windows
+    // cut from the first key not yet covered.  Query block qb takes key u of
+    // block b iff bit u % 64 of rw[qb - b] is set, so lane `lane` holds, for
+    // its block b and each query block, the words of blocks b and b + 1; a
+    // window starting at bit s of block b takes bits s.. of the first and
+    // bits ..s-1 of the second.  Each 64-key word starts at most one window.
+    // (Windows cut per slot instead, from each slot's own keys, double the
+    // chunk stream and measured slower.)
+    if (ranges) {
+        long long cursor = 0;  // keys below it lie in an emitted window
+        for (int base = 0; base <= bmax && pr.ok; base += 32) {
+            const int b = base + lane;
+            uint64_t lo[4], hi[4], nb = 0;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int dl = qb0 + qq - b;
+                lo[qq] = (qq < nqb && b <= bmax && dl >= 0) ? rw[dl] : 0ull;
+                hi[qq] = (qq < nqb && b + 1 <= bmax && dl >= 1) ? rw[dl - 1] : 0ull;
+                nb |= lo[qq];
+            }
+            unsigned bal = __ballot_sync(0xffffffffu, nb != 0ull);
+            while (bal && pr.ok) {
+                const int src = __ffs(bal) - 1;
+                bal &= bal - 1;
+                const long long kb = 64LL * (base + src);
+                uint64_t bits = __shfl_sync(0xffffffffu, nb, src);
+                const long long c = cursor - kb;
+                if (c >= 64) bits = 0ull;
+                else if (c > 0) bits &= ~0ull << c;
+                if (!bits) continue;  // covered by the window before
+                const int sft = __ffsll((long long)bits) - 1;
+                uint64_t qm[4];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const uint64_t a = __shfl_sync(0xffffffffu, lo[qq], src);
+                    const uint64_t h = __shfl_sync(0xffffffffu, hi[qq], src);
+                    qm[qq] = (a >> sft) | (sft ? h << (64 - sft) : 0ull);
+                }
+                pr.window((int)(kb + sft), qm);
+                cursor = kb + sft + 64;
+            }
+        }
+    }
+
     // --- 64-key blocks, ascending, one chunk each
-    for (int base = 0; base <= bmax && pr.ok; base += 32) {
+    for (int base = 0; base <= bmax && pr.ok && !ranges; base += 32) {
         const int b = base + lane;
         int m = 0;
         if (b <= bmax) {
@@ -481,7 +569,9 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tmQ, const 
                     const int qb = qb0 + qq;
                     if (j < 64 * (qb + 1)) {
                         const int delta = qb - (j >> 6);
-                        if (!bit_of(patmap, delta)) m |= 1 << qq;
+                        const bool covered =
+                            ranges ? ((rw[delta] >> (j & 63)) & 1ull) != 0 : bit_of(patmap, delta);
+                        if (!covered) m |= 1 << qq;
                     }
                 }
             }
@@ -701,6 +791,8 @@ __device__ void run_softmax(const AttnParams& p, uint8_t* sm, const Bars& bars,
             uint64_t keep = ~0ull;
             unsigned kv = 1u;  // bit 0: some row of the warp takes the chunk; bit 1: some row drops a key
             if (d.info & kChunkWhole) {
+            } else if (type == kChunkRange) {
+                keep = d.qmask[qi] & low_bits(i - (long long)d.b + 1);  // and causal
             } else if (type == kChunkBlock) {
                 keep = 0;
                 if ((d.m >> qi) & 1) {
@@ -967,18 +1059,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Per VS head: slash offsets -> block-diagonal bitmap D (offset o touches
 // deltas o/64 and, unless o % 64 == 0, o/64 + 1), vertical columns -> sorted
 // unique list.  Entries outside [0, N) other than the -1 padding are counted.
+//
+// With `ranges`, also the range words of the range reading of a diagonal
+// (diagonal o gives query block bq the keys 64 bq - o .. 64 bq + 63 - o):
+// query block bq takes key u iff some selected o lies in
+// [64 bq - u, 64 bq - u + 63], which depends only on delta = bq - u / 64 and
+// i = u % 64.  rwords[delta] holds that as bit i:
+//   bit i of rwords[delta] = some selected o in [64 delta - i, 64 delta - i + 63].
 __global__ void __launch_bounds__(1024) vs_prep_kernel(const int32_t* __restrict__ v_idx,
                                                        int kv_stride, int kv,
                                                        const int32_t* __restrict__ s_idx,
                                                        int ks_stride, int ks, int N,
-                                                       VsPrepWs ws, int32_t* err) {
+                                                       VsPrepWs ws, int32_t* err, bool ranges) {
     extern __shared__ uint32_t dsm[];
     __shared__ int warp_tot[33];
     const int pos = blockIdx.x;
     const int nB = N / 64, nBw = (nB + 31) / 32, nW = N / 32;
     uint32_t* col = ws.colbits + (size_t)pos * nW;
+    uint32_t* sb = ws.sbits + (size_t)pos * nW;
     for (int w = threadIdx.x; w < nBw; w += blockDim.x) dsm[w] = 0;
     for (int w = threadIdx.x; w < nW; w += blockDim.x) col[w] = 0;
+    if (ranges)
+        for (int w = threadIdx.x; w < nW; w += blockDim.x) sb[w] = 0;
     __syncthreads();
     for (int t = threadIdx.x; t < ks; t += blockDim.x) {
         const int o = s_idx[(size_t)pos * ks_stride + t];
@@ -989,6 +1091,7 @@ __global__ void __launch_bounds__(1024) vs_prep_kernel(const int32_t* __restrict
         const int a = o >> 6;
         atomicOr(&dsm[a >> 5], 1u << (a & 31));
         if ((o & 63) && a + 1 < nB) atomicOr(&dsm[(a + 1) >> 5], 1u << ((a + 1) & 31));
+        if (ranges) atomicOr(&sb[o >> 5], 1u << (o & 31));
     }
     for (int t = threadIdx.x; t < kv; t += blockDim.x) {
         const int j = v_idx[(size_t)pos * kv_stride + t];
@@ -1000,6 +1103,21 @@ __global__ void __launch_bounds__(1024) vs_prep_kernel(const int32_t* __restrict
     }
     __syncthreads();
     for (int w = threadIdx.x; w < nBw; w += blockDim.x) ws.dbits[(size_t)pos * nBw + w] = dsm[w];
+    if (ranges) {
+        // 64-bit words of the offset bitmap: word t holds offsets 64 t .. 64 t + 63
+        const uint64_t* s64 = reinterpret_cast<const uint64_t*>(sb);
+        uint64_t* rw = ws.rwords + (size_t)pos * nB;
+        for (int dl = threadIdx.x; dl < nB; dl += blockDim.x) {
+            const uint64_t a = dl > 0 ? s64[dl - 1] : 0ull;  // offsets 64 dl - 64 .. 64 dl - 1
+            const uint64_t b = s64[dl];                      // offsets 64 dl .. 64 dl + 63
+            uint64_t w = b != 0ull ? 1ull : 0ull;
+            // i >= 1: offsets 64 dl - i .. 64 dl - 1 are the top i bits of a,
+            // offsets 64 dl .. 64 dl + 63 - i the low 64 - i bits of b
+            for (int i = 1; i < 64; ++i)
+                if ((a >> (64 - i)) != 0ull || (b << i) != 0ull) w |= 1ull << i;
+            rw[dl] = w;
+        }
+    }
     // ordered compaction of the column bitmap
     int32_t* out = ws.vlist + (size_t)pos * ws.vcap;
     int base_out = 0;
@@ -1067,6 +1185,7 @@ cudaError_t launch_attn_d(const AttnLaunch& a, cudaStream_t st) {
     p.n_super = (a.N + 255) / 256;
     p.scale_log2 = (float)(a.scale * 1.4426950408889634);
     p.dbits = a.dbits;
+    p.rwords = a.rwords;
     p.nBw = (p.nB + 31) / 32;
     p.vlist = a.vlist;
     p.vcnt = a.vcnt;
@@ -1143,6 +1262,8 @@ VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv) {
     if (w.vcap < 1) w.vcap = 1;
     w.dbits = c.take<uint32_t>((size_t)n_heads * nBw);
     w.colbits = c.take<uint32_t>((size_t)n_heads * (N / 32));
+    w.sbits = c.take<uint32_t>((size_t)n_heads * (N / 32));
+    w.rwords = c.take<uint64_t>((size_t)n_heads * nB);
     w.vlist = c.take<int32_t>((size_t)n_heads * w.vcap);
     w.vcnt = c.take<int32_t>((size_t)n_heads);
     return w;
@@ -1150,11 +1271,11 @@ VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv) {
 
 cudaError_t launch_vs_prep(const int32_t* v_idx, int kv_stride, int kv, const int32_t* s_idx,
                            int ks_stride, int ks, int N, int n_heads, const VsPrepWs& ws,
-                           int32_t* err_count, cudaStream_t st) {
+                           int32_t* err_count, cudaStream_t st, bool ranges) {
     if (n_heads == 0) return cudaSuccess;
     const int nBw = (N / 64 + 31) / 32;
-    vs_prep_kernel<<<n_heads, 1024, nBw * sizeof(uint32_t), st>>>(v_idx, kv_stride, kv, s_idx,
-                                                                  ks_stride, ks, N, ws, err_count);
+    vs_prep_kernel<<<n_heads, 1024, nBw * sizeof(uint32_t), st>>>(
+        v_idx, kv_stride, kv, s_idx, ks_stride, ks, N, ws, err_count, ranges);
     return cudaGetLastError();
 }
 

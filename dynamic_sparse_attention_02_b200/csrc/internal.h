@@ -14,8 +14,9 @@ namespace minfer {
 using bf16 = __nv_bfloat16;
 
 // Query heads of one launch, in list order.  Each entry packs
-// qh (bits 0-11), pattern (bits 12-13) and the head's position in the
-// per-pattern index arrays (bits 16-31).
+// qh (bits 0-11), pattern (bits 12-13), the Vertical-Slash range flag (bit 14:
+// slash diagonals as unaligned 64-key ranges instead of 64x64 tiles) and the
+// head's position in the per-pattern index arrays (bits 16-31).
 struct HeadList {
     int n;
     uint32_t e[MI_MAX_HEADS];
@@ -26,6 +27,10 @@ __host__ __device__ inline uint32_t pack_head(int qh, int pattern, int pidx) {
 }
 __host__ __device__ inline int head_qh(uint32_t e) { return (int)(e & 0xFFFu); }
 __host__ __device__ inline int head_pattern(uint32_t e) { return (int)((e >> 12) & 0x3u); }
+__host__ __device__ inline bool head_ranges(uint32_t e) { return ((e >> 14) & 1u) != 0; }
+__host__ __device__ inline uint32_t with_ranges(uint32_t e, bool on) {
+    return on ? (e | (1u << 14)) : (e & ~(1u << 14));
+}
 __host__ __device__ inline int head_pidx(uint32_t e) { return (int)(e >> 16); }
 // grouped-query attention, contiguous groups
 __host__ __device__ inline int kv_head_of(int qh, int Hq, int Hkv) {
@@ -105,14 +110,18 @@ cudaError_t launch_bs_index(const bf16* q, const bf16* k, int Hq, int Hkv, int N
 struct VsPrepWs {
     uint32_t* dbits;    // [n_heads][nBw]   slash diagonals -> block-diagonal set
     uint32_t* colbits;  // [n_heads][N/32]  vertical columns as a bitmap
+    uint32_t* sbits;    // [n_heads][N/32]  slash offsets as a bitmap
+    uint64_t* rwords;   // [n_heads][nB]    range words (see vs_prep_kernel)
     int32_t* vlist;     // [n_heads][vcap]  sorted unique columns
     int32_t* vcnt;      // [n_heads]
     int vcap;
 };
 VsPrepWs carve_vs_prep(WsCarver& c, int n_heads, int N, int kv);
+// ranges: also build the range words (needed by heads whose slash diagonals
+// select unaligned 64-key ranges)
 cudaError_t launch_vs_prep(const int32_t* v_idx, int kv_stride, int kv, const int32_t* s_idx,
                            int ks_stride, int ks, int N, int n_heads, const VsPrepWs& ws,
-                           int32_t* err_count, cudaStream_t st);
+                           int32_t* err_count, cudaStream_t st, bool ranges = false);
 
 struct AttnLaunch {
     const bf16 *q, *k, *v;
@@ -121,8 +130,9 @@ struct AttnLaunch {
     int Hq, Hkv, N, d;
     double scale;
     HeadList heads;  // pattern + per-pattern position per entry
-    // Vertical-Slash
+    // Vertical-Slash (rwords: range words, read by heads with the range flag)
     const uint32_t* dbits;
+    const uint64_t* rwords;
     const int32_t* vlist;
     const int32_t* vcnt;
     int vcap;

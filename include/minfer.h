@@ -83,6 +83,15 @@ enum {
 #define MI_MAX_HEADS 256
 #define MI_BLOCK 64
 
+/* How a Vertical-Slash head's selected diagonals become attended keys:
+ *  MI_SLASH_BLOCKS -- every 64x64 tile a diagonal touches is computed whole
+ *    (the tile lists of the guide's "Vertical-Slash Kernel Mechanics");
+ *  MI_SLASH_RANGES -- diagonal o gives query block bq (rows 64 bq .. 64 bq + 63)
+ *    the 64 keys 64 bq - o .. 64 bq + 63 - o, causally masked: the keys
+ *    its rows reach along the diagonal, as one unaligned range per block
+ *    (fewer keys than the tiles; see mi_vs_range_attn). */
+enum { MI_SLASH_BLOCKS = 0, MI_SLASH_RANGES = 1 };
+
 /* Per-pattern parameters of one layer (all heads of a pattern share them). */
 typedef struct {
     int last_q;        /* VS: number of final queries that score columns/diagonals */
@@ -91,6 +100,7 @@ typedef struct {
     int topk_blocks;   /* BS: key blocks kept per 64-row query block */
     int sink;          /* A-shape: keys 0..sink-1 always kept */
     int window;        /* A-shape: keys i-window+1 .. i kept for row i */
+    int slash_tiles;   /* VS: MI_SLASH_BLOCKS (0, the default) or MI_SLASH_RANGES */
 } mi_params;
 
 /* Stage boundaries recorded by mi_prefill_layer when stage_events != NULL:
@@ -181,6 +191,26 @@ int mi_vs_sparse_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int 
                       const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
                       mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
                       void* stream);
+
+/*
+ * Vertical-Slash sparse attention with range slash tiles (MI_SLASH_RANGES):
+ * the guide's cost model for this pattern ("2. The Vertical-Slash Pattern":
+ * work in proportion to the kept columns and diagonals) with the diagonals
+ * streamed as contiguous key runs ("Vertical-Slash Kernel Mechanics").
+ * Row i of query block bq = i / 64 attends key j <= i iff j is one of the
+ * head's vertical columns, or some selected diagonal o has
+ * 64 bq - o <= j <= 64 bq + 63 - o.  The kept keys of a block are a union
+ * of such 64-key runs; the kernel covers it with 64-key tiles that start at
+ * any key, so an isolated diagonal costs one tile per query block instead of
+ * the two 64x64 tiles it touches.  Arguments, layouts, workspace
+ * (mi_workspace_bytes with MI_OP_VS_ATTN) and errors as for
+ * mi_vs_sparse_attn.
+ */
+int mi_vs_range_attn(const mi_bf16* q, const mi_bf16* k, const mi_bf16* v, int Hq, int Hkv,
+                     int N, int d, float scale, const int32_t* v_idx, int vertical_size,
+                     const int32_t* s_idx, int slash_size, const int32_t* heads, int n_heads,
+                     mi_bf16* out, float* lse, int32_t* err_count, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /*
  * Block-sparse attention (guide, "3. The Block-Sparse Pattern": only the

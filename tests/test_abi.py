@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = header_functions()
-    assert len(names) == 18
+    assert len(names) == 19
     assert sorted(B.EXPORTS) == names
     for n in names:
         assert hasattr(lib, n), n
@@ -148,6 +148,14 @@ def test_prefill_layer_heads_validation(lib):
                                       ctypes.cast(arr, ctypes.c_void_p), f, None, None, f,
                                       1 << 30, None, None) == B.MI_ERR_INVALID_ARG
     assert B.mi_prefill_workspace_bytes_heads(4, 2, 512, 128, pat, ps) == 0
+    ps[1] = B.make_params(slash_tiles=2)                 # neither tiles nor ranges
+    arr = (B.mi_params * 4)(*ps)
+    assert lib.mi_prefill_layer_heads(f, f, f, 4, 2, 512, 128, 0.0,
+                                      pat.ctypes.data_as(ctypes.c_void_p),
+                                      ctypes.cast(arr, ctypes.c_void_p), f, None, None, f,
+                                      1 << 30, None, None) == B.MI_ERR_INVALID_ARG
+    ps[1] = B.make_params(slash_tiles=B.MI_SLASH_RANGES)  # one range head: a valid plan
+    assert B.mi_prefill_workspace_bytes_heads(4, 2, 512, 128, pat, ps) > 0
     ps[1] = B.make_params()
     ps[3] = B.make_params(window=0)                      # A-shape window >= 1
     arr = (B.mi_params * 4)(*ps)
@@ -155,6 +163,22 @@ def test_prefill_layer_heads_validation(lib):
                                       pat.ctypes.data_as(ctypes.c_void_p),
                                       ctypes.cast(arr, ctypes.c_void_p), f, None, None, f,
                                       1 << 30, None, None) == B.MI_ERR_INVALID_ARG
+
+
+def test_vs_range_attn_validation(lib):
+    f = FAKE
+    args = [f, f, f, 4, 2, 512, 128, 0.0, f, 16, f, 32, None, 0, f, None, None]
+    ws = B.mi_workspace_bytes(B.MI_OP_VS_ATTN, 4, 2, 512, 128, 0, 0, 16, 32)
+    assert lib.mi_vs_range_attn(*args, f, ws - 256, None) == B.MI_ERR_WORKSPACE
+    bad = list(args)
+    bad[0] = None
+    assert lib.mi_vs_range_attn(*bad, f, ws, None) == B.MI_ERR_INVALID_ARG
+    bad = list(args)
+    bad[3] = 3                                            # Hq % Hkv
+    assert lib.mi_vs_range_attn(*bad, f, ws, None) == B.MI_ERR_INVALID_ARG
+    bad = list(args)
+    bad[5] = 500                                          # N % 64
+    assert lib.mi_vs_range_attn(*bad, f, ws, None) == B.MI_ERR_UNSUPPORTED
 
 
 def test_workspace_queries(lib):
