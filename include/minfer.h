@@ -316,9 +316,11 @@ int mi_vs_index_static(const mi_bf16* q, const mi_bf16* k, int Hq, int Hkv, int 
  * 3 MMA/stage-full, 4 MMA/P-ready, 5 softmax/stage-full, 6 softmax/S-ready,
  * 7 softmax/O-done) and 11..15 for the score passes (11 producer/stage-free,
  * 12 MMA/Q, 13 MMA/stage-full, 14 MMA/accumulator-free, 15 epilogue/
- * accumulator-full); site 0 means no wait gave up.  Attention's record is
- * returned when it holds one, else the score passes'.  Reading copies the
- * record to `record8` (host int32 [8]) and clears both.  A correct run never
+ * accumulator-full), and 21..27 for the key-major Block-Sparse engine
+ * (21 producer, 22-24 MMA issue, 25-27 softmax); site 0 means no wait
+ * gave up.  The row-major attention record is returned when it holds one,
+ * else the key-major one, else the score passes'.  Reading copies the record
+ * to `record8` (host int32 [8]) and clears all three.  A correct run never
  * records anything.
  */
 int mi_debug_wait_failure(int32_t* record8);
