@@ -27,6 +27,34 @@ def test_vs_useful_flops_matches_brute_force():
             assert bench.vs_useful_flops(v, s, N, 128) == brute(v, s, N, 128)
 
 
+def brute_range(v_idx, s_idx, N, d):
+    """Range reading, from the oracle's element mask: per query block, the kept
+    slash keys (seen by the block's last row) as runs, each run of n keys
+    costing ceil(n / 64) tiles; gathered columns are the kept columns outside
+    the block's slash keys."""
+    nB = N // 64
+    s = np.asarray([x for x in s_idx if 0 <= x < N], np.int32)
+    v = np.asarray(sorted(set(int(x) for x in v_idx if 0 <= x < N)), np.int32)
+    ms = oracle.vs_mask(N, np.zeros(0, np.int32), s, range_tiles=True)
+    tiles = cols = 0
+    for bq in range(nB):
+        row = ms[64 * bq + 63].astype(np.int8)
+        m = np.diff(np.concatenate([[0], row, [0]]))
+        st, en = np.nonzero(m == 1)[0], np.nonzero(m == -1)[0]
+        tiles += int(np.sum((en - st + 63) // 64))
+        cols += int(np.sum(~ms[64 * bq + 63, v[v <= 64 * bq + 63]]))
+    return 4.0 * d * (64 * 64 * tiles + 64 * cols), tiles, cols
+
+
+def test_vs_range_useful_flops_matches_the_oracle_mask():
+    rng = np.random.default_rng(1)
+    for N in (512, 1024, 1600):
+        for _ in range(4):
+            v = rng.integers(-1, N, size=rng.integers(0, 40)).astype(np.int32)
+            s = rng.integers(-1, N, size=rng.integers(1, 30)).astype(np.int32)
+            assert bench.vs_range_useful_flops(v, s, N, 128) == brute_range(v, s, N, 128)
+
+
 def test_ashape_tile_count_matches_brute_force():
     """The closed-form count of 64x64 tiles an A-shape head computes (bench FLOP
     accounting) equals a direct count over every causal (query block, key block)."""
