@@ -93,11 +93,38 @@ def params_of(w, B, ranges=False):
                          slash_tiles=B.MI_SLASH_RANGES if ranges else B.MI_SLASH_BLOCKS)
 
 
+def _code_only(src):
+    """C/C++ source with comments and whitespace removed (string literals kept),
+    so that a comment edit does not orphan measurements taken on the code."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c == '"' or c == "'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            if not c.isspace():
+                out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def attn_source_sha():
+    """Hash of the attention kernel's code (comments and whitespace ignored): the
+    key under which ncu records of that kernel are kept."""
     h = hashlib.sha256()
     for name in ATTN_SOURCES:
-        with open(os.path.join(ROOT, "dynamic_sparse_attention_02_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "dynamic_sparse_attention_02_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

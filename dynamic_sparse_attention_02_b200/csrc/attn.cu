@@ -10,13 +10,15 @@
 //
 // Work item = one query head x one 256-row "super tile" (four 64-row query
 // blocks), held as two 128-row slots.  The producer enumerates the item's
-// key chunks -- one 64-key block, or up to 64 gathered vertical columns --
-// each with a 4-bit mask (one bit per query block); a chunk is computed for
-// the slots whose bits it carries.  Each softmax row turns the descriptor
-// into a 64-bit mask of the keys it takes (causal limit, A-shape sink and
-// window, gathered columns); a warp whose query block does not take the
-// chunk writes zero P rows and skips the exponentials, and chunks that every
-// row takes whole are flagged so that they skip the mask step.
+// key chunks -- one 64-key block, 64 consecutive keys from any offset (a
+// Vertical-Slash head that reads its diagonals as ranges), or up to 64
+// gathered vertical columns -- each with a 4-bit mask (one bit per query
+// block); a chunk is computed for the slots whose bits it carries.  Each
+// softmax row turns the descriptor into a 64-bit mask of the keys it takes
+// (causal limit, A-shape sink and window, gathered columns, a range chunk's
+// keys per query block); a warp whose query block does not take the chunk
+// writes zero P rows and skips the exponentials, and chunks that every row
+// takes whole are flagged so that they skip the mask step.
 //   warps 0-3  softmax, slot 0 (TMEM lanes 0-127 = rows 0-127)
 //   warps 4-7  softmax, slot 1 (rows 128-255)
 //   warp 8     producer: chunk list + TMA loads (cp.async gathers), 4 deep

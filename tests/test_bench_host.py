@@ -120,3 +120,13 @@ def test_reference_arm_json_line(capsys, monkeypatch):
     assert "2048 seeded random rows" in cb["sample"]  # the whole small layer was sampled
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_code_only_hash_ignores_comments_not_code():
+    a = 'int f() { // one\n  return 1; /* two */ }\nconst char* s = "// kept";\n'
+    b = 'int f() {   // other words\n return 1; }\n/* c */ const char* s = "// kept";'
+    c = 'int f() { return 2; }\nconst char* s = "// kept";'
+    d = 'int f() { return 1; }\nconst char* s = "// other";'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert bench._code_only(a) != bench._code_only(d)

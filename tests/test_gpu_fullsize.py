@@ -29,10 +29,11 @@ def _built():
     build.build()
 
 
-def run_layer(w):
+def run_layer(w, ranges=False):
     x = synth.make_inputs(w, device="cuda")
     p = B.make_params(last_q=w.last_q, vertical_size=w.vertical_size, slash_size=w.slash_size,
-                      topk_blocks=w.topk_blocks, sink=w.sink, window=w.window)
+                      topk_blocks=w.topk_blocks, sink=w.sink, window=w.window,
+                      slash_tiles=B.MI_SLASH_RANGES if ranges else B.MI_SLASH_BLOCKS)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, lse = B.mi_prefill_layer(x["q"], x["k"], x["v"], x["pattern"], p, want_lse=True,
                                   err_count=err)
@@ -41,7 +42,7 @@ def run_layer(w):
     return x, out, lse
 
 
-def check_head(w, x, out_layer, lse_layer, h, rows):
+def check_head(w, x, out_layer, lse_layer, h, rows, ranges=False):
     q, k, v = x["q"], x["k"], x["v"]
     qs, ks_, vs_ = head_slices(q, k, v, h)
     pt = int(x["pattern"][h])
@@ -54,14 +55,15 @@ def check_head(w, x, out_layer, lse_layer, h, rows):
         gva, gsa = gv[0].cpu().numpy(), gs[0].cpu().numpy()
         same_index &= check_index_set(gva, vert, w.vertical_size, what=f"vertical h{h}") == 0
         same_index &= check_index_set(gsa, sl, w.slash_size, what=f"slash h{h}") == 0
-        ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, a, b, rows=rows)
+        attn_ref = oracle.attn_vs_range if ranges else oracle.attn_vs
+        ro, rl = attn_ref(qs, ks_, vs_, 0, a, b, rows=rows)
         if not same_index:
-            layer_ref = oracle.attn_vs(qs, ks_, vs_, 0, gva[gva >= 0], gsa[gsa >= 0], rows=rows)
+            layer_ref = attn_ref(qs, ks_, vs_, 0, gva[gva >= 0], gsa[gsa >= 0], rows=rows)
         vi = torch.full((1, w.vertical_size), -1, dtype=torch.int32)
         si = torch.full((1, w.slash_size), -1, dtype=torch.int32)
         vi[0, :a.size] = torch.from_numpy(a.astype(np.int32))
         si[0, :b.size] = torch.from_numpy(b.astype(np.int32))
-        out, lse = B.mi_vs_sparse_attn(q, k, v, vi.cuda(), si.cuda(), heads=[h])
+        out, lse = B.mi_vs_sparse_attn(q, k, v, vi.cuda(), si.cuda(), heads=[h], ranges=ranges)
     elif pt == synth.PATTERN_BS:
         bi, bc, S = oracle.bs_index(qs, ks_, 0, w.topk_blocks, want_scores=True)
         gbi, gbc = B.mi_bs_index(q, k, w.topk_blocks, heads=[h])
@@ -112,5 +114,39 @@ def test_full_size_layer_matches_oracle(name, n_heads, n_rows):
         heads = sorted(set(heads) | set(extra))
     ties = [h for h in heads if not check_head(w, x, out, lse, h, rows)]
     print(f"{name}: {len(heads)} heads checked, {len(ties)} with index ties {ties}")
+    del x, out, lse
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,n_heads,n_rows", [
+    ("vs_n128k_llama3_8b", 2, 256),
+    ("vs_n1m_llama3_8b", 2, 1024),
+])
+def test_full_size_range_tiles_match_oracle(name, n_heads, n_rows):
+    """The same layers with every Vertical-Slash head reading its diagonals as
+    64-key ranges (MI_SLASH_RANGES), against the oracle's range reading."""
+    w = synth.workload(name)
+    x, out, lse = run_layer(w, ranges=True)
+    assert torch.isfinite(out.float()).all()
+    heads, rows = synth.sample_heads_rows(w, n_heads, n_rows, seed=w.seed + 1)
+    ties = [h for h in heads if not check_head(w, x, out, lse, h, rows, ranges=True)]
+    print(f"{name} (ranges): {len(heads)} heads checked, {len(ties)} with index ties {ties}")
+    del x, out, lse
+    torch.cuda.empty_cache()
+
+
+def test_full_size_block_sparse_on_the_key_major_engine():
+    """The 128K Block-Sparse layer with Block-Sparse heads on the key-major
+    engine (mi_set_bs_engine), against the oracle on sampled heads and rows."""
+    w = synth.workload("bs_n128k_llama3_8b")
+    B.mi_set_bs_engine(B.BS_ENGINE_KEY)
+    try:
+        x, out, lse = run_layer(w)
+        assert torch.isfinite(out.float()).all()
+        heads, rows = synth.sample_heads_rows(w, 2, 256, seed=w.seed + 2)
+        ties = [h for h in heads if not check_head(w, x, out, lse, h, rows)]
+    finally:
+        B.mi_set_bs_engine(B.BS_ENGINE_ROW)
+    print(f"bs_n128k (key-major): {len(heads)} heads checked, {len(ties)} with index ties {ties}")
     del x, out, lse
     torch.cuda.empty_cache()
