@@ -129,11 +129,12 @@ def test_bs_index_head_subset():
 
 def _attn_call(which, q, k, v, heads, out, lse, ws):
     N = q.shape[1]
-    if which == "vs":
+    if which in ("vs", "vs_range"):
         vi = torch.tensor([[0, 5, 300, N - 1, -1]] * len(heads), dtype=torch.int32,
                           device="cuda")
         si = torch.tensor([[0, 64, 200, -1]] * len(heads), dtype=torch.int32, device="cuda")
-        B.mi_vs_sparse_attn(q, k, v, vi, si, heads=heads, out=out, lse=lse, ws=ws)
+        B.mi_vs_sparse_attn(q, k, v, vi, si, heads=heads, out=out, lse=lse, ws=ws,
+                            ranges=which == "vs_range")
     elif which in ("bs", "bs_key"):
         nB = N // 64
         bi = torch.full((len(heads), nB, 3), -1, dtype=torch.int32, device="cuda")
@@ -153,14 +154,14 @@ def _attn_call(which, q, k, v, heads, out, lse, ws):
         B.mi_dense_attn(q, k, v, heads=heads, out=out, lse=lse)
 
 
-@pytest.mark.parametrize("which", ["vs", "bs", "bs_key", "ashape", "dense"])
+@pytest.mark.parametrize("which", ["vs", "vs_range", "bs", "bs_key", "ashape", "dense"])
 def test_attention_touches_listed_heads_only(which):
     Hq, Hkv, N, d = 6, 2, 640, 128
     q, k, v = rand_bf16(Hq, Hkv, N, d, 43)
     heads = [5, 0, 2]
     out, lse = Guarded((Hq, N, d), torch.bfloat16), Guarded((Hq, N), torch.float32)
     ws = None
-    if which == "vs":
+    if which in ("vs", "vs_range"):
         nb = B.mi_workspace_bytes(B.MI_OP_VS_ATTN, Hq, Hkv, N, d, len(heads), 0, 5)
         raw, ws = workspace(nb)
     _attn_call(which, q, k, v, heads, out.view, lse.view, ws)

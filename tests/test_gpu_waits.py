@@ -23,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 ATTN_SITES = range(1, 8)    # producer / MMA / softmax waits of the attention kernel
 SCORE_SITES = range(11, 16)  # producer / MMA / epilogue waits of the VS score passes
+KT_SITES = range(21, 28)     # producer / MMA / softmax waits of the key-major engine
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -68,6 +69,43 @@ def test_attention_wait_gives_up_then_device_is_usable():
         qs, ks_, vs_ = head_slices(q, k, v, h)
         ro, rl = oracle.attn_vs(qs, ks_, vs_, 0, vi[h].cpu().numpy(), si[h].cpu().numpy())
         check_attn(out[h], lse[h], ro, rl, what=f"after the give-up, head {h}")
+    assert B.mi_debug_wait_failure()["site"] == 0
+
+
+def test_key_major_engine_wait_gives_up_then_device_is_usable():
+    """The same for the key-major Block-Sparse engine (sites 21-27)."""
+    Hq, Hkv, N, d, topk = 2, 1, 1024, 128, 6
+    q, k, v = rand_bf16(Hq, Hkv, N, d, 53)
+    bi = np.full((Hq, N // 64, topk), -1, np.int32)
+    bc = np.zeros((Hq, N // 64), np.int32)
+    for h in range(Hq):
+        qs, ks_, _ = head_slices(q, k, None, h)
+        bi[h], bc[h] = oracle.bs_index(qs, ks_, 0, topk)
+    bit, bct = torch.from_numpy(bi).cuda(), torch.from_numpy(bc).cuda()
+    B.mi_debug_wait_failure()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    B.mi_set_bs_engine(B.BS_ENGINE_KEY)
+    try:
+        B.mi_debug_set_wait_budget(1)
+        try:
+            out, lse = B.mi_block_sparse_attn(q, k, v, bit, bct, err_count=err)
+            torch.cuda.synchronize()
+        finally:
+            B.mi_debug_set_wait_budget(0)
+        assert int(err.item()) & (1 << 30), "no wait gave up with a one-cycle budget"
+        rec = B.mi_debug_wait_failure()
+        assert rec["site"] in KT_SITES, rec
+        assert torch.isfinite(out.float()).all()
+        err.zero_()
+        out, lse = B.mi_block_sparse_attn(q, k, v, bit, bct, err_count=err)
+        torch.cuda.synchronize()
+    finally:
+        B.mi_set_bs_engine(B.BS_ENGINE_ROW)
+    assert int(err.item()) == 0
+    for h in range(Hq):
+        qs, ks_, vs_ = head_slices(q, k, v, h)
+        ro, rl = oracle.attn_bs(qs, ks_, vs_, 0, bi[h], bc[h])
+        check_attn(out[h], lse[h], ro, rl, what=f"key-major after the give-up, head {h}")
     assert B.mi_debug_wait_failure()["site"] == 0
 
 
