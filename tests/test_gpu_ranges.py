@@ -161,3 +161,21 @@ def test_prefill_layer_all_range_heads_one_params():
         a, b, _, _ = oracle.vs_index(qs, ks_, 0, 64, 100, 200)
         ro, rl = oracle.attn_vs_range(qs, ks_, vs_, 0, a, b)
         check_attn(out[h], lse[h], ro, rl, what=f"all-range layer h{h}")
+
+
+@pytest.mark.parametrize("N,d,si,vi", [
+    (64, 128, [0, 5, 63], [-1]),            # one block: every range starts at or before key 0
+    (192, 64, [191, 1, 64], [100]),         # the last diagonal reaches key 0 of the last block only
+    (320, 128, [130, 129, 128, 127], []),   # four adjacent diagonals merge into one run
+    (256, 128, [-1, -1], [0, 255]),         # no diagonal: the verticals alone
+])
+def test_vs_range_attn_small_edges(N, d, si, vi):
+    q, k, v = rand_bf16(1, 1, N, d, 74)
+    s = np.array([si], np.int32)
+    c = np.array([vi if vi else [-1]], np.int32)
+    out, lse = B.mi_vs_sparse_attn(q, k, v, torch.from_numpy(c).cuda(), torch.from_numpy(s).cuda(),
+                                   ranges=True)
+    torch.cuda.synchronize()
+    qs, ks_, vs_ = head_slices(q, k, v, 0)
+    ro, rl = oracle.attn_vs_range(qs, ks_, vs_, 0, c[0][c[0] >= 0], s[0][s[0] >= 0])
+    check_attn(out[0], lse[0], ro, rl, what=f"range edge N={N}")
